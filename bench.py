@@ -1,0 +1,530 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A16 group-32 mixture-of-experts layer on B200.
+
+Default workload: one MoE decode layer with 64 tokens, 128 experts, top-8 routing, hidden 2816,
+expert intermediate 704 (gate/up int4 [128, 1408, 2816], down int4 [128, 2816, 704], group 32,
+bf16 scales).  A step is one pass of the hot path: route + permute, gate/up grouped GEMM with the
+GELU gate, down grouped GEMM, weighted combine.  Metric: tokens per second (higher is better).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                  [--workload moe_decode|moe_prefill] [--no-secondary]
+
+Multi-GPU: the layer does not shard in this build; N ranks run N independent replicas (weak
+scaling), timed on the device with the max over ranks.  `--impl reference` times the CPU oracle
+(the correctness reference) on the same workload, one token per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE W4A16 grouped-GEMM tokens/s; achieved HBM GB/s / TC util vs B200 peak"
+UNIT = "tokens/s"
+
+WORKLOADS = {
+    "moe_decode": dict(T=64, zipf=None, name="moe_decode_T64_E128_top8_H2816_I704_g32"),
+    "moe_prefill": dict(T=8192, zipf=1.1, name="moe_prefill_T8192_E128_top8_H2816_I704_g32_zipf1.1"),
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default="moe_decode")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------------------------------
+# distributed plumbing
+# ------------------------------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu_index), "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, which):
+        if which == "begin":
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self):
+        time.sleep(0.25)
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            rows.append((ts, parts))
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        inside = [r for r in rows if self.t0 is not None and self.t0 - 0.15 <= r[0] <= (self.t1 or r[0]) + 0.15]
+        use = inside if inside else rows
+        sm = [float(p[1]) for _, p in use if p[1].replace(".", "").isdigit()]
+        smax = [float(p[2]) for _, p in use if p[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for _, p in use:
+            for name, v in zip(names, p[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(use),
+                "power_w_max": max((float(p[3]) for _, p in use if p[3].replace(".", "").isdigit()), default=None)}
+
+
+# ------------------------------------------------------------------------------------------
+# native arm
+# ------------------------------------------------------------------------------------------
+
+def to_dev(a, kind, device):
+    import numpy as np
+    import torch
+    if kind == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+    if kind == "u32":
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int32)).to(device)
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+
+
+def gmm_bytes(counts, T, k, H, I):
+    """Algorithmic bytes of the two grouped GEMM launches: codes + scales of every expert that
+    received a token, activations read once, outputs written once."""
+    hit = int((counts > 0).sum())
+    gu_w = 2 * I * (H // 8) * 4 + 2 * I * (H // 32) * 2
+    dn_w = H * (I // 8) * 4 + H * (I // 32) * 2
+    gu = hit * gu_w + T * H * 2 + T * k * I * 2
+    dn = hit * dn_w + T * k * I * 2 + T * k * H * 2
+    return gu, dn, hit
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    p = os.path.join(ROOT, "w4a16_group_quantized_w4_b200", "csrc", "stream_gemm.cu")
+    h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def read_profile_traffic(name):
+    """dram bytes per launch from a committed ncu summary, if taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        if ":" in line and line.strip().startswith("- "):
+            k, _, v = line.strip()[2:].partition(":")
+            vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def native(args, world, rank, local):
+    import numpy as np
+    import torch
+
+    from w4a16_group_quantized_w4_b200 import api, synth
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    wl = WORKLOADS[args.workload]
+    T, E, k, H, I = wl["T"], 128, 8, 2816, 704
+    case = synth.moe_case(T, E, k, H, I, seed=args.seed + rank, zipf_s=wl["zipf"])
+    copies = 2
+    layers = []
+    for c in range(copies):
+        layers.append(api.MoELayer(to_dev(case.gu_codes, "u32", device), to_dev(case.gu_scales, "bf16", device),
+                                   to_dev(case.dn_codes, "u32", device), to_dev(case.dn_scales, "bf16", device), T, k))
+    x = to_dev(case.x, "bf16", device)
+    logits = to_dev(case.logits, "f32", device)
+    stream = torch.cuda.Stream(device)
+    torch.cuda.synchronize()
+
+    # warm-up, then capture one step per weight copy into CUDA graphs
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            layers[i % copies](x, logits)
+    stream.synchronize()
+    graphs = []
+    for c in range(copies):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            layers[c](x, logits)
+        graphs.append(g)
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            graphs[i % copies].replay()
+    stream.synchronize()
+
+    # ---------------- timed region (device step, graph replay) ----------------
+    gpu_index = _physical_gpu_index(local)
+    clocks = ClockSampler(gpu_index)
+    clocks.start()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    clocks.mark("begin")
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for i in range(args.steps):
+            graphs[i % copies].replay()
+        ev1.record(stream)
+    stream.synchronize()
+    clocks.mark("end")
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    clocks.stop()
+    ms_per_step = ms / args.steps
+    value = T * world * args.steps / (ms / 1e3)
+
+    # ---------------- per-kernel durations of the grouped GEMM (same launches) ----------------
+    lay = layers[0]
+    gu_c, gu_s, dn_c, dn_s = lay.w
+    n_k = min(300, args.steps)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_k)]
+    with torch.cuda.stream(stream):
+        api.moe_route_permute(logits, k, out=lay.rt, ws=lay.route_ws)
+        for i in range(n_k):
+            e0, e1, e2 = evs[i]
+            e0.record(stream)
+            api.moe_w4a16_gmm(x, lay.rt.sorted_pair, k, gu_c, gu_s, lay.rt.expert_offsets, T * k,
+                              api.W4_EPI_GELU_GATE, out=lay.h)
+            e1.record(stream)
+            api.moe_w4a16_gmm(lay.h, None, 1, dn_c, dn_s, lay.rt.expert_offsets, T * k,
+                              api.W4_EPI_NONE, out=lay.o)
+            e2.record(stream)
+    stream.synchronize()
+    t_gu = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(n_k)) / 1e3
+    t_dn = statistics.mean(evs[i][1].elapsed_time(evs[i][2]) for i in range(n_k)) / 1e3
+    counts = np.diff(lay.rt.expert_offsets.cpu().numpy())
+    b_gu, b_dn, hit = gmm_bytes(counts, T, k, H, I)
+    hbm_peak, tc_peak, tc_sus, peak_src = peaks()
+    achieved = (b_gu + b_dn) / (t_gu + t_dn) / 1e9
+    traffic = read_profile_traffic(f"stream_gemm_{args.workload}.md")
+
+    # ---------------- end to end through the public API with host buffers ----------------
+    x_h = torch.empty_like(x, device="cpu").pin_memory()
+    x_h.copy_(x.cpu())
+    lg_h = torch.empty_like(logits, device="cpu").pin_memory()
+    lg_h.copy_(logits.cpu())
+    y_h = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(x)
+    lg_d = torch.empty_like(logits)
+    n_e2e = min(args.steps, 500)
+    with torch.cuda.stream(stream):
+        for _ in range(5):
+            x_d.copy_(x_h, non_blocking=True)
+            lg_d.copy_(lg_h, non_blocking=True)
+            y = lay(x_d, lg_d)
+            y_h.copy_(y, non_blocking=True)
+    stream.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for _ in range(n_e2e):
+            x_d.copy_(x_h, non_blocking=True)
+            lg_d.copy_(lg_h, non_blocking=True)
+            y = lay(x_d, lg_d)
+            y_h.copy_(y, non_blocking=True)
+        f1.record(stream)
+    stream.synchronize()
+    ms_e2e = f0.elapsed_time(f1)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms_e2e], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    e2e_value = T * world * n_e2e / (ms_e2e / 1e3)
+
+    secondary = {}
+    if not args.no_secondary and rank == 0:
+        secondary = run_secondary(args, device, stream)
+
+    cpu_base = None
+    if rank == 0 and world == 1:
+        cpu_base = cpu_baseline(case)
+
+    if world > 1:
+        import torch.distributed as dist
+        del graphs
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded: codes uniform over -8..7, scales 0.01|N(0,1)|+1e-4, x and logits N(0,1))",
+        "config": {"workload": wl["name"], "tokens_per_step": T, "experts": E, "top_k": k,
+                   "hidden": H, "intermediate": I, "group": 32, "parallelism": f"replicas{world}",
+                   "l2": f"no flush: {copies} weight copies of 428 MB alternate, each step streams the "
+                         f"{hit} experts hit (>126 MB L2)",
+                   "timing": "CUDA graph replay of the 4-launch step, CUDA events on the launch stream"},
+        "clocks": clocks.summary(),
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT,
+                "h2d_bytes_per_step": int(x.numel() * 2 + logits.numel() * 4),
+                "d2h_bytes_per_step": int(T * H * 2),
+                "how": "public API (MoELayer) per step: pinned H2D of x and logits, 4 launches, D2H of y"},
+        "gpu_launches": 4 * args.steps,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                     "kernel": "stream_gemm_kernel (gate/up + down launches of one step)",
+                     "algorithmic_bytes_per_step": int(b_gu + b_dn), "experts_hit": hit,
+                     "us_gate_up": round(t_gu * 1e6, 2), "us_down": round(t_dn * 1e6, 2),
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"},
+        "cpu_baseline": cpu_base,
+        "secondary": secondary,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _physical_gpu_index(local):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        items = [v.strip() for v in vis.split(",") if v.strip()]
+        if local < len(items) and items[local].isdigit():
+            return int(items[local])
+    return local
+
+
+def cpu_baseline(case):
+    """The oracle as it stands on a bounded sample of the same workload (host cores)."""
+    import numpy as np
+
+    from oracle import moe
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=os.cpu_count())
+    except Exception:
+        threads = os.cpu_count()
+    tokens = np.arange(16)
+    t0 = time.perf_counter()
+    moe.moe_layer(case.x, case.logits, case.gu_codes, case.gu_scales, case.dn_codes, case.dn_scales,
+                  case.k, tokens=tokens)
+    dt = time.perf_counter() - t0
+    return {"value": round(len(tokens) / dt, 3), "unit": UNIT, "cores": int(threads), "kind": "oracle",
+            "sample": f"{len(tokens)} of {case.T} tokens of the same layer (routing of all {case.T}); "
+                      f"{dt:.1f} s of float64 numpy on the host"}
+
+
+def run_secondary(args, device, stream):
+    """Other configurations of the same kernels, timed briefly (not the headline)."""
+    import numpy as np
+    import torch
+
+    from w4a16_group_quantized_w4_b200 import api, synth
+    out = {}
+    hbm_peak, _, _, _ = peaks()
+    # dense decode GEMV, K=4096, N=14336: 8 rotating weight copies (264 MB > 2x L2)
+    base = synth.case_dense_gemv(16)
+    nc = 8
+    codes = [to_dev(base.codes, "u32", device) for _ in range(nc)]
+    scales = [to_dev(base.scales, "bf16", device) for _ in range(nc)]
+    for M in (1, 4, 16):
+        xx = to_dev(base.x[:M], "bf16", device)
+        yy = torch.empty((M, 14336), dtype=torch.bfloat16, device=device)
+        with torch.cuda.stream(stream):
+            for i in range(10):
+                api.w4a16_linear(xx, codes[i % nc], scales[i % nc], y=yy)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(nc):
+                    api.w4a16_linear(xx, codes[i], scales[i], y=yy)
+            g.replay()
+        stream.synchronize()
+        reps = 50
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (reps * nc)
+        byts = 14336 * 4096 // 2 + 14336 * 128 * 2 + M * 4096 * 2 + M * 14336 * 2
+        out[f"dense_gemv_M{M}_K4096_N14336"] = {"us": round(us, 2), "GB/s": round(byts / us / 1e3, 1),
+                                                 "frac_hbm": round(byts / us / 1e3 / hbm_peak, 3)}
+        del g
+    del codes, scales
+    torch.cuda.empty_cache()
+    # MoE prefill layer (8192 tokens, Zipf-skewed experts), a few steps
+    if args.workload != "moe_prefill":
+        pc = synth.case_moe_prefill(args.seed)
+        lay = api.MoELayer(to_dev(pc.gu_codes, "u32", device), to_dev(pc.gu_scales, "bf16", device),
+                           to_dev(pc.dn_codes, "u32", device), to_dev(pc.dn_scales, "bf16", device),
+                           pc.T, pc.k)
+        xx, ll = to_dev(pc.x, "bf16", device), to_dev(pc.logits, "f32", device)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                lay(xx, ll)
+        stream.synchronize()
+        reps = 5
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                lay(xx, ll)
+            e1.record(stream)
+        stream.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        flops = 2.0 * pc.T * pc.k * (2 * 704 * 2816 + 2816 * 704)
+        _, tc_peak, _, _ = peaks()
+        out["moe_prefill_T8192_zipf1.1"] = {"ms": round(ms, 3), "tokens/s": round(pc.T / ms * 1e3, 1),
+                                            "TFLOP/s": round(flops / ms / 1e9, 1),
+                                            "frac_bf16_peak": round(flops / ms / 1e9 / tc_peak, 3)}
+        del lay
+        torch.cuda.empty_cache()
+    return out
+
+
+# ------------------------------------------------------------------------------------------
+# reference arm: the CPU oracle on the same workload
+# ------------------------------------------------------------------------------------------
+
+def reference(args, world, rank):
+    if rank != 0:
+        return
+    import numpy as np
+
+    from oracle import moe
+    from w4a16_group_quantized_w4_b200 import synth
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=os.cpu_count())
+    except Exception:
+        threads = os.cpu_count()
+    wl = WORKLOADS[args.workload]
+    case = synth.moe_case(wl["T"], 128, 8, 2816, 704, seed=args.seed, zipf_s=wl["zipf"])
+    budget_s = 150.0
+
+    def step(i):
+        t = i % case.T
+        moe.moe_layer(case.x, case.logits, case.gu_codes, case.gu_scales, case.dn_codes,
+                      case.dn_scales, case.k, tokens=[t])
+
+    t0 = time.perf_counter()
+    step(0)
+    one = time.perf_counter() - t0
+    n_w = min(args.warmup, max(0, int(0.1 * budget_s / one)))
+    for i in range(n_w):
+        step(i)
+    n_run = max(1, min(args.steps, int(0.9 * budget_s / one)))
+    t0 = time.perf_counter()
+    for i in range(n_run):
+        step(i)
+    dt = time.perf_counter() - t0
+    value = n_run / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+        "steps": n_run, "steps_requested": args.steps, "warmup": n_w, "ms_per_step": round(dt / n_run * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same seeded inputs as the native arm)",
+        "config": {"workload": wl["name"], "tokens_per_step": 1, "experts": 128, "top_k": 8,
+                   "hidden": 2816, "intermediate": 704, "group": 32, "parallelism": "host"},
+        "cpu_baseline": {"kind": "oracle", "cores": int(threads), "value": round(value, 4), "unit": UNIT,
+                         "sample": f"one token of the {case.T}-token layer per step (its 8 expert pairs), "
+                                   f"steps capped to a {budget_s:.0f} s budget"},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        reference(args, world, rank)
+        return
+    native(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,79 @@
+"""GPU parity of w4a16_linear against the float64 oracle.
+
+Definition: "Repacked QAT Gemma 4 26B-A4B serves on one TPU v6e at 1.9x FP8 throughput", section
+"What changed in vLLM's TPU backend" (W4A16 linear: per-32 scales, weights dequantised on chip,
+bf16 activations).  Tolerance per output row: rel-L2 <= 5e-3 and max-abs <= 2e-2 * max|y_ref|;
+the exact-integer case is compared bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import bf16, linear, q4
+from w4a16_group_quantized_w4_b200 import api, synth
+from tests._util import assert_rows_close, dev_bf16, dev_u32, host_bf16_bits, host_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(case):
+    y = api.w4a16_linear(dev_bf16(case.x), dev_u32(case.codes), dev_bf16(case.scales))
+    torch.cuda.synchronize()
+    return y
+
+
+def test_dense_small_config():
+    case = synth.case_dense_small()
+    ref = linear.w4a16_linear(case.x, case.codes, case.scales)
+    assert_rows_close(host_f64(_run(case)), ref)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 32), (3, 13, 96), (5, 200, 256), (16, 64, 2816),
+                                   (33, 136, 704), (64, 256, 512), (100, 128, 4096), (1, 1, 64)])
+def test_ragged_shapes(M, N, K):
+    case = synth.dense_case(M, N, K, 0.02, 1e-3, seed=M * 7 + N)
+    ref = linear.w4a16_linear(case.x, case.codes, case.scales)
+    assert_rows_close(host_f64(_run(case)), ref)
+
+
+def test_exact_integer_case_bit_exact():
+    """x with at most 16 nonzero entries of +-1 per row and power-of-two scales: y is an integer
+    multiple of a power of two below 2^8 in magnitude, so bf16 holds it exactly."""
+    rng = np.random.default_rng(31)
+    M, N, K = 8, 384, 1024
+    x = np.zeros((M, K), np.float32)
+    for m in range(M):
+        idx = rng.choice(K, size=16, replace=False)
+        x[m, idx] = rng.choice([-1.0, 1.0], size=16)
+    q = rng.integers(-8, 8, size=(N, K))
+    s = np.full((N, K // 32), 0.125, np.float32)
+    x_bits = synth.f32_to_bf16_bits(x)
+    codes = q4.pack(q)
+    s_bits = synth.f32_to_bf16_bits(s)
+    ref = linear.w4a16_linear(x_bits, codes, s_bits)
+    y = api.w4a16_linear(dev_bf16(x_bits), dev_u32(codes), dev_bf16(s_bits))
+    assert np.array_equal(host_bf16_bits(y), bf16.from_f64(ref))
+
+
+def test_zero_rows():
+    case = synth.dense_case(0, 64, 256, 0.02, 1e-3, seed=1)
+    y = api.w4a16_linear(dev_bf16(case.x), dev_u32(case.codes), dev_bf16(case.scales))
+    assert y.shape == (0, 64)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_decode_gemv_full_size_sampled(M):
+    """K=4096, N=14336 at full size; 160 sampled output columns checked against the oracle."""
+    case = synth.case_dense_gemv(M)
+    y = host_f64(_run(case))
+    rng = np.random.default_rng(M)
+    cols = np.unique(np.concatenate([[0, 127, 128, 14335], rng.choice(14336, 156, replace=False)]))
+    ref = linear.w4a16_linear_rows(case.x, case.codes, case.scales, cols)
+    assert_rows_close(y[:, cols], ref)
+
+
+def test_repeat_calls_are_deterministic():
+    case = synth.case_dense_gemv(4)
+    y1 = host_bf16_bits(_run(case))
+    y2 = host_bf16_bits(_run(case))
+    assert np.array_equal(y1, y2)

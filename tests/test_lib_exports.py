@@ -1,0 +1,57 @@
+"""The C-ABI library loads and exports every entry point include/w4a16.h declares (CPU only).
+
+Also checks host-side argument validation, which returns before any CUDA call.
+"""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from w4a16_group_quantized_w4_b200 import _lib
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "w4a16.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                       text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for must in ("w4_repack", "w4a16_linear", "moe_route_permute", "moe_w4a16_gmm", "moe_combine",
+                 "w4_workspace_bytes", "w4_status_str", "w4_last_cuda_error"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported():
+    lib = _lib.load()
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert set(_declared()) <= set(_lib.SIGNATURES)
+
+
+def test_host_validation_rejects_bad_arguments():
+    lib = _lib.load()
+    nul = C.c_void_p(None)
+    bogus = C.c_void_p(16)
+    assert lib.w4_repack(bogus, 4, 33, bogus, bogus, nul, nul, nul) == _lib.W4_ERR_INVALID_ARG
+    assert lib.w4_repack(nul, 4, 64, bogus, bogus, nul, nul, nul) == _lib.W4_ERR_INVALID_ARG
+    assert lib.w4a16_linear(bogus, bogus, bogus, bogus, 1, 0, 64, nul, 0, nul) == _lib.W4_ERR_INVALID_ARG
+    assert lib.w4a16_linear(C.c_void_p(18), bogus, bogus, bogus, 1, 8, 64, nul, 0, nul) == _lib.W4_ERR_INVALID_ARG
+    assert lib.moe_route_permute(bogus, 4, 128, 0, bogus, bogus, bogus, bogus, bogus, nul, 0, nul) == _lib.W4_ERR_INVALID_ARG
+    assert lib.moe_route_permute(bogus, 4, 2000, 8, bogus, bogus, bogus, bogus, bogus, nul, 0, nul) == _lib.W4_ERR_INVALID_ARG
+    assert lib.moe_w4a16_gmm(bogus, nul, 1, bogus, bogus, bogus, 8, 16, 63, 64, 1, bogus, nul, 0, nul, nul) == _lib.W4_ERR_INVALID_ARG
+    assert lib.moe_w4a16_gmm(bogus, nul, 1, bogus, bogus, bogus, 8, 16, 64, 64, 7, bogus, nul, 0, nul, nul) == _lib.W4_ERR_INVALID_ARG
+    assert lib.moe_combine(bogus, bogus, bogus, 4, 8, 12, bogus, nul) == _lib.W4_ERR_INVALID_ARG
+    assert lib.w4_status_str(_lib.W4_ERR_TIMEOUT) == b"W4_ERR_TIMEOUT"
+    assert lib.w4_workspace_bytes(99, 1, 1, 32, 1, 1) == 0
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError):
+        _lib.load(str(tmp_path / "nope.so"))

@@ -1,0 +1,155 @@
+// C ABI of libw4a16: argument checks, dispatch to the kernels, workspace sizing, status text.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/w4a16.h"
+
+// kernel launchers (repack.cu, route.cu, stream_gemm.cu)
+w4_status w4_launch_repack(const uint16_t* w, int64_t groups, uint32_t* codes, uint16_t* scales,
+                           uint8_t* group_m, unsigned long long* off_grid_count,
+                           cudaStream_t stream, int sm_count);
+size_t w4_route_workspace_bytes(int T, int E);
+w4_status w4_launch_route(const float* logits, int T, int E, int k, int32_t* ids, float* w,
+                          int32_t* offsets, int32_t* sorted_pair, int32_t* pair_pos, void* ws,
+                          size_t ws_bytes, cudaStream_t stream);
+w4_status w4_launch_combine(const uint16_t* o, const float* topk_w, const int32_t* pair_pos, int T,
+                            int k, int H, uint16_t* y, cudaStream_t stream);
+size_t w4_stream_workspace_bytes(int64_t rows, int N, int K, int E, int epi, bool dense, int sm_count);
+w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int k_div,
+                                const uint32_t* codes, const uint16_t* scales,
+                                const int32_t* offsets, int E, int64_t rows, int N, int K, int epi,
+                                uint16_t* out, void* ws, size_t ws_bytes, int32_t* dev_status,
+                                cudaStream_t stream, int sm_count);
+
+namespace {
+
+thread_local int32_t g_last_cuda_error = 0;
+
+int current_sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 64 && cached[dev]) return cached[dev];
+  int n = 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev < 64) cached[dev] = n;
+  return n;
+}
+
+// Returns the status and records the CUDA error behind a W4_ERR_CUDA.
+w4_status finish(w4_status s) {
+  if (s == W4_ERR_CUDA) {
+    cudaError_t e = cudaGetLastError();
+    g_last_cuda_error = static_cast<int32_t>(e == cudaSuccess ? cudaErrorUnknown : e);
+  }
+  return s;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+const char* w4_status_str(int32_t s) {
+  switch (s) {
+    case W4_OK: return "W4_OK";
+    case W4_ERR_INVALID_ARG: return "W4_ERR_INVALID_ARG";
+    case W4_ERR_UNSUPPORTED: return "W4_ERR_UNSUPPORTED";
+    case W4_ERR_CUDA: return "W4_ERR_CUDA";
+    case W4_ERR_TIMEOUT: return "W4_ERR_TIMEOUT";
+    case W4_ERR_WORKSPACE: return "W4_ERR_WORKSPACE";
+    default: return "W4_ERR_UNKNOWN";
+  }
+}
+
+int32_t w4_last_cuda_error(void) { return g_last_cuda_error; }
+
+size_t w4_workspace_bytes(int32_t op, int64_t M_or_T, int64_t N, int64_t K, int32_t E, int32_t k) {
+  (void)k;
+  if (M_or_T < 0 || N < 0 || K < 0 || E < 0) return 0;
+  switch (op) {
+    case W4_OP_LINEAR:
+      if (N <= 0 || K < 32 || K % 32) return 0;
+      return w4_stream_workspace_bytes(M_or_T, static_cast<int>(N), static_cast<int>(K), 1,
+                                       W4_EPI_NONE, true, current_sm_count());
+    case W4_OP_ROUTE:
+      return w4_route_workspace_bytes(static_cast<int>(M_or_T), E);
+    case W4_OP_GMM:
+      return 0;
+    default:
+      return 0;
+  }
+}
+
+w4_status w4_repack(const uint16_t* w, int64_t rows, int64_t K, uint32_t* codes, uint16_t* scales,
+                    uint8_t* group_m, unsigned long long* off_grid_count, void* stream) {
+  if (rows < 0 || K < 32 || K % 32) return W4_ERR_INVALID_ARG;
+  if (rows > 0 && (!w || !codes || !scales)) return W4_ERR_INVALID_ARG;
+  if ((w && !aligned(w, 16)) || (codes && !aligned(codes, 16)) || (scales && !aligned(scales, 2)))
+    return W4_ERR_INVALID_ARG;
+  if (off_grid_count && !aligned(off_grid_count, 8)) return W4_ERR_INVALID_ARG;
+  const int64_t groups = rows * (K / 32);
+  return finish(w4_launch_repack(w, groups, codes, scales, group_m, off_grid_count,
+                                 static_cast<cudaStream_t>(stream), current_sm_count()));
+}
+
+w4_status w4a16_linear(const uint16_t* x, const uint32_t* codes, const uint16_t* scales,
+                       uint16_t* y, int64_t M, int64_t N, int64_t K, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  if (M < 0 || N < 1 || K < 32 || K % 32 || N > (1LL << 30) || K > (1LL << 30)) return W4_ERR_INVALID_ARG;
+  if (M > 0 && (!x || !y)) return W4_ERR_INVALID_ARG;
+  if (!codes || !scales) return W4_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(scales, 4) || (x && !aligned(x, 16)) || (y && !aligned(y, 16)))
+    return W4_ERR_INVALID_ARG;
+  if (workspace && !aligned(workspace, 16)) return W4_ERR_INVALID_ARG;
+  if (M * N > (1LL << 40)) return W4_ERR_UNSUPPORTED;
+  return finish(w4_launch_stream_gemm(x, nullptr, 1, codes, scales, nullptr, 1, M,
+                                      static_cast<int>(N), static_cast<int>(K), W4_EPI_NONE, y,
+                                      workspace, workspace_bytes, nullptr,
+                                      static_cast<cudaStream_t>(stream), current_sm_count()));
+}
+
+w4_status moe_route_permute(const float* logits, int32_t T, int32_t E, int32_t k, int32_t* topk_ids,
+                            float* topk_w, int32_t* expert_offsets, int32_t* sorted_pair,
+                            int32_t* pair_pos, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (T < 0 || E < 1 || E > 1024 || k < 1 || k > 32 || k > E) return W4_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(T) * k > (1LL << 30)) return W4_ERR_UNSUPPORTED;
+  if (!expert_offsets) return W4_ERR_INVALID_ARG;
+  if (T > 0 && (!logits || !topk_ids || !topk_w || !sorted_pair || !pair_pos)) return W4_ERR_INVALID_ARG;
+  return finish(w4_launch_route(logits, T, E, k, topk_ids, topk_w, expert_offsets, sorted_pair,
+                                pair_pos, workspace, workspace_bytes,
+                                static_cast<cudaStream_t>(stream)));
+}
+
+w4_status moe_w4a16_gmm(const uint16_t* a, const int32_t* a_row_of_pair, int32_t k,
+                        const uint32_t* codes, const uint16_t* scales, const int32_t* expert_offsets,
+                        int32_t E, int64_t rows, int32_t N, int32_t K, int32_t epilogue,
+                        uint16_t* out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                        void* stream) {
+  if (E < 1 || E > 1024 || rows < 0 || N < 1 || K < 32 || K % 32) return W4_ERR_INVALID_ARG;
+  if (epilogue != W4_EPI_NONE && epilogue != W4_EPI_GELU_GATE) return W4_ERR_INVALID_ARG;
+  if (epilogue == W4_EPI_GELU_GATE && (N % 2)) return W4_ERR_INVALID_ARG;
+  if (a_row_of_pair && k < 1) return W4_ERR_INVALID_ARG;
+  if (!codes || !scales || !expert_offsets) return W4_ERR_INVALID_ARG;
+  if (rows > 0 && (!a || !out)) return W4_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(scales, 4) || (a && !aligned(a, 16)) || (out && !aligned(out, 16)))
+    return W4_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(E) * N > (1LL << 31) - 1 || rows > (1LL << 31) - 1) return W4_ERR_UNSUPPORTED;
+  return finish(w4_launch_stream_gemm(a, a_row_of_pair, k, codes, scales, expert_offsets, E, rows, N,
+                                      K, epilogue, out, workspace, workspace_bytes, dev_status,
+                                      static_cast<cudaStream_t>(stream), current_sm_count()));
+}
+
+w4_status moe_combine(const uint16_t* o, const float* topk_w, const int32_t* pair_pos, int32_t T,
+                      int32_t k, int32_t H, uint16_t* y, void* stream) {
+  if (T < 0 || k < 1 || H < 8 || H % 8) return W4_ERR_INVALID_ARG;
+  if (T > 0 && (!o || !topk_w || !pair_pos || !y)) return W4_ERR_INVALID_ARG;
+  if ((o && !aligned(o, 16)) || (y && !aligned(y, 16))) return W4_ERR_INVALID_ARG;
+  return finish(w4_launch_combine(o, topk_w, pair_pos, T, k, H, y, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

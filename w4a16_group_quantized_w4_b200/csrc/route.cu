@@ -1,0 +1,297 @@
+// Top-k routing, softmax weights and the stable expert-major permutation.
+//
+// The pages give 128 experts per layer with 8 active per token ("Repacked QAT Gemma 4 26B-A4B
+// serves on one TPU v6e at 1.9x FP8 throughput", section "The gap at 26B"); the selection rule
+// (largest logits, equal logits by lower index, descending), softmax over the selected, and the
+// (expert, pair id) order of the permutation are the definitions stated in w4a16.h.
+//
+// Mapping:
+//   topk     one warp per token.  The lane holding expert e keeps its logits in registers; k rounds
+//            of a warp-wide arg-max (value, then lower index) pick the winners.  Lanes 0..k-1 then
+//            form the softmax with one exp each and a warp sum.  Per-CTA expert histograms go to
+//            the workspace.
+//   scatter  every CTA re-derives the global counts and its own base per expert from all CTAs'
+//            histograms (deterministic, no atomics on positions), CTA 0 writes expert_offsets,
+//            and each warp walks a contiguous run of pairs: a per-warp histogram pass, a scan of
+//            the warp bases, then positions from __match_any_sync ranks.  Positions are exact and
+//            independent of scheduling.
+//   Small T runs both phases in one CTA (one launch); large T uses two launches.
+#include "common.cuh"
+
+namespace w4 {
+
+constexpr int kRouteWarps = 8;                 // warps per CTA
+constexpr int kRouteTokensPerCta = 64;         // tokens per CTA in the two-launch path
+constexpr int kMaxEPerLane = 32;               // E <= 1024
+
+struct RouteArgs {
+  const float* logits;
+  int T, E, k;
+  int32_t* topk_ids;
+  float* topk_w;
+  int32_t* expert_offsets;
+  int32_t* sorted_pair;
+  int32_t* pair_pos;
+  int32_t* hist;       // [num_ctas][E] per-CTA counts (workspace)
+  int tokens_per_cta;
+};
+
+__device__ __forceinline__ bool better(float v, int i, float w, int j) {
+  return v > w || (v == w && i < j);
+}
+
+// Top-k for tokens [t0, t1) of this CTA; accumulates counts into s_cnt[E] (shared).
+__device__ void topk_tokens(const RouteArgs& A, int t0, int t1, int* s_cnt) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int per_lane = (A.E + 31) >> 5;
+  for (int t = t0 + warp; t < t1; t += nwarps) {
+    float v[kMaxEPerLane];
+    const float* row = A.logits + static_cast<int64_t>(t) * A.E;
+#pragma unroll
+    for (int c = 0; c < kMaxEPerLane; ++c) {
+      const int e = c * 32 + lane;
+      v[c] = (c < per_lane && e < A.E) ? row[e] : -INFINITY;
+    }
+    uint32_t taken = 0;
+    float sel_v = 0.f;
+    int sel_e = 0;
+    float top = 0.f;
+    for (int j = 0; j < A.k; ++j) {
+      float bv = -INFINITY;
+      int be = 0x7FFFFFFF;
+#pragma unroll
+      for (int c = 0; c < kMaxEPerLane; ++c) {
+        const int e = c * 32 + lane;
+        if (c < per_lane && e < A.E && !((taken >> c) & 1u) && better(v[c], e, bv, be)) {
+          bv = v[c];
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (better(ov, oe, bv, be)) { bv = ov; be = oe; }
+      }
+      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      if (j == 0) top = bv;
+      if (lane == j) { sel_v = bv; sel_e = be; }
+    }
+    const float ex = lane < A.k ? expf(sel_v - top) : 0.f;
+    float sum = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane < A.k) {
+      A.topk_ids[static_cast<int64_t>(t) * A.k + lane] = sel_e;
+      A.topk_w[static_cast<int64_t>(t) * A.k + lane] = ex / sum;
+      atomicAdd(&s_cnt[sel_e], 1);
+    }
+  }
+}
+
+// Positions for pairs [p0, p1) given this CTA's per-expert base s_base[E] (shared).
+// s_wcnt: [nwarps][E] shared scratch.
+__device__ void scatter_pairs(const RouteArgs& A, int64_t p0, int64_t p1, const int* s_base,
+                              int* s_wcnt) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int64_t n = p1 - p0;
+  const int64_t per_warp = (n + nwarps - 1) / nwarps;
+  const int64_t w0 = p0 + warp * per_warp;
+  const int64_t w1 = min(p1, w0 + per_warp);
+  int* mycnt = s_wcnt + warp * A.E;
+  for (int e = lane; e < A.E; e += 32) mycnt[e] = 0;
+  __syncwarp();
+  for (int64_t p = w0 + lane; p - lane < w1; p += 32) {
+    int e = p < w1 ? A.topk_ids[p] : -1;
+    if (e >= A.E) e = -1;
+    const bool valid = e >= 0;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int leader = __ffs(peers) - 1;
+    if (valid && lane == leader) mycnt[e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // exclusive scan over warps per expert: base for warp w = s_base[e] + sum_{w' < w} cnt[w'][e]
+  for (int e = threadIdx.x; e < A.E; e += blockDim.x) {
+    int run = s_base[e];
+    for (int w = 0; w < nwarps; ++w) {
+      const int c = s_wcnt[w * A.E + e];
+      s_wcnt[w * A.E + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  for (int64_t p = w0 + lane; p - lane < w1; p += 32) {
+    int e = p < w1 ? A.topk_ids[p] : -1;
+    if (e >= A.E) e = -1;
+    const bool valid = e >= 0;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const unsigned lt = peers & ((1u << lane) - 1u);
+    if (valid) {
+      const int pos = mycnt[e] + __popc(lt);
+      if (pos >= 0 && static_cast<int64_t>(pos) < static_cast<int64_t>(A.T) * A.k) {
+        A.sorted_pair[pos] = static_cast<int32_t>(p);
+        A.pair_pos[p] = pos;
+      }
+    }
+    __syncwarp();
+    const int leader = __ffs(peers) - 1;
+    if (valid && lane == leader) mycnt[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+// One CTA does everything (small T).
+__global__ void __launch_bounds__(kRouteWarps * 32) route_fused_kernel(RouteArgs A) {
+  extern __shared__ int smem[];
+  int* s_cnt = smem;                     // [E]
+  int* s_base = s_cnt + A.E;             // [E]
+  int* s_wcnt = s_base + A.E;            // [nwarps][E]
+  for (int e = threadIdx.x; e < A.E; e += blockDim.x) s_cnt[e] = 0;
+  __syncthreads();
+  topk_tokens(A, 0, A.T, s_cnt);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int e = 0; e < A.E; ++e) {
+      s_base[e] = run;
+      A.expert_offsets[e] = run;
+      run += s_cnt[e];
+    }
+    A.expert_offsets[A.E] = run;
+  }
+  __syncthreads();
+  __threadfence_block();
+  scatter_pairs(A, 0, static_cast<int64_t>(A.T) * A.k, s_base, s_wcnt);
+}
+
+__global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(RouteArgs A) {
+  extern __shared__ int smem[];
+  int* s_cnt = smem;
+  for (int e = threadIdx.x; e < A.E; e += blockDim.x) s_cnt[e] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * A.tokens_per_cta;
+  const int t1 = min(A.T, t0 + A.tokens_per_cta);
+  topk_tokens(A, t0, t1, s_cnt);
+  __syncthreads();
+  for (int e = threadIdx.x; e < A.E; e += blockDim.x) A.hist[blockIdx.x * A.E + e] = s_cnt[e];
+}
+
+__global__ void __launch_bounds__(kRouteWarps * 32) route_scatter_kernel(RouteArgs A) {
+  extern __shared__ int smem[];
+  int* s_tot = smem;                     // [E]
+  int* s_base = s_tot + A.E;             // [E]
+  int* s_wcnt = s_base + A.E;            // [nwarps][E]
+  const int nctas = gridDim.x;
+  for (int e = threadIdx.x; e < A.E; e += blockDim.x) {
+    int tot = 0, mine = 0;
+    for (int c = 0; c < nctas; ++c) {
+      const int v = A.hist[c * A.E + e];
+      if (c < static_cast<int>(blockIdx.x)) mine += v;
+      tot += v;
+    }
+    s_tot[e] = tot;
+    s_base[e] = mine;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int e = 0; e < A.E; ++e) {
+      const int t = s_tot[e];
+      s_tot[e] = run;          // exclusive prefix = expert offset
+      run += t;
+    }
+    if (blockIdx.x == 0) A.expert_offsets[A.E] = run;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < A.E; e += blockDim.x) {
+    if (blockIdx.x == 0) A.expert_offsets[e] = s_tot[e];
+    s_base[e] += s_tot[e];
+  }
+  __syncthreads();
+  const int64_t p0 = static_cast<int64_t>(blockIdx.x) * A.tokens_per_cta * A.k;
+  const int64_t p1 = min(static_cast<int64_t>(A.T) * A.k, p0 + static_cast<int64_t>(A.tokens_per_cta) * A.k);
+  scatter_pairs(A, p0, p1, s_base, s_wcnt);
+}
+
+// ------------------------------------------------------------------------------------------
+// combine: y[t] = sum_j w[t, j] * o[pair_pos[t*k + j]], float32 in slot order, bf16 out.
+// One thread per 8 consecutive features (16-byte loads and stores).
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) combine_kernel(const uint16_t* __restrict__ o,
+                                                      const float* __restrict__ topk_w,
+                                                      const int32_t* __restrict__ pair_pos,
+                                                      int T, int k, int H, uint16_t* __restrict__ y) {
+  const int t = blockIdx.x;
+  const int h8 = blockIdx.y * blockDim.x + threadIdx.x;
+  if (t >= T || h8 * 8 >= H) return;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int j = 0; j < k; ++j) {
+    const float wj = topk_w[static_cast<int64_t>(t) * k + j];
+    const int64_t row = pair_pos[static_cast<int64_t>(t) * k + j];
+    if (row < 0 || row >= static_cast<int64_t>(T) * k) continue;   // not a valid permutation entry
+    const uint4 v = ldg_stream128(o + row * H + h8 * 8);
+    const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[2 * i] = fmaf(wj, bf16_lo_to_f32(vv[i]), acc[2 * i]);
+      acc[2 * i + 1] = fmaf(wj, bf16_hi_to_f32(vv[i]), acc[2 * i + 1]);
+    }
+  }
+  uint4 out;
+  out.x = pack_bf16x2(acc[0], acc[1]);
+  out.y = pack_bf16x2(acc[2], acc[3]);
+  out.z = pack_bf16x2(acc[4], acc[5]);
+  out.w = pack_bf16x2(acc[6], acc[7]);
+  *reinterpret_cast<uint4*>(y + static_cast<int64_t>(t) * H + h8 * 8) = out;
+}
+
+}  // namespace w4
+
+// ---------------------------------------------------------------------------------------------
+// host launchers (declared in api.cu)
+// ---------------------------------------------------------------------------------------------
+
+static int route_num_ctas(int T) { return (T + w4::kRouteTokensPerCta - 1) / w4::kRouteTokensPerCta; }
+
+size_t w4_route_workspace_bytes(int T, int E) {
+  if (T <= w4::kRouteTokensPerCta * 4) return 0;   // fused single-CTA path
+  return static_cast<size_t>(route_num_ctas(T)) * E * sizeof(int32_t);
+}
+
+w4_status w4_launch_route(const float* logits, int T, int E, int k, int32_t* ids, float* w,
+                          int32_t* offsets, int32_t* sorted_pair, int32_t* pair_pos, void* ws,
+                          size_t ws_bytes, cudaStream_t stream) {
+  w4::RouteArgs A{logits, T, E, k, ids, w, offsets, sorted_pair, pair_pos, nullptr,
+                  w4::kRouteTokensPerCta};
+  const int threads = w4::kRouteWarps * 32;
+  const size_t smem = static_cast<size_t>(2 + w4::kRouteWarps) * E * sizeof(int);
+  // (2 + warps) * E ints <= 40 KB for E <= 1024: within the default shared-memory limit
+  if (T == 0) {
+    // offsets are all zero
+    if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), stream) != cudaSuccess) return W4_ERR_CUDA;
+    return W4_OK;
+  }
+  if (w4_route_workspace_bytes(T, E) == 0) {
+    w4::route_fused_kernel<<<1, threads, smem, stream>>>(A);
+  } else {
+    if (ws == nullptr || ws_bytes < w4_route_workspace_bytes(T, E)) return W4_ERR_WORKSPACE;
+    A.hist = static_cast<int32_t*>(ws);
+    const int nctas = route_num_ctas(T);
+    w4::route_topk_kernel<<<nctas, threads, E * sizeof(int), stream>>>(A);
+    if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
+    w4::route_scatter_kernel<<<nctas, threads, smem, stream>>>(A);
+  }
+  return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+w4_status w4_launch_combine(const uint16_t* o, const float* topk_w, const int32_t* pair_pos, int T,
+                            int k, int H, uint16_t* y, cudaStream_t stream) {
+  if (T == 0) return W4_OK;
+  const int threads = 128;
+  dim3 grid(T, (H / 8 + threads - 1) / threads);
+  w4::combine_kernel<<<grid, threads, 0, stream>>>(o, topk_w, pair_pos, T, k, H, y);
+  return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
