@@ -23,9 +23,10 @@ Readings taken where the pages are open (each is also listed in the design notes
     off the grid with codes 0 and a NaN scale.
 
 Packed layout (ours; the container's bit layout is not on the pages): codes[r, w] is a uint32
-whose bits 4j..4j+3 hold u = q + 8 of element k = 8w + j (low nibble = lower k).  One 16-byte
-run of four words is exactly one group of 32.  Scales[r, g] is the bf16 scale of elements
-32g..32g+31 of row r.
+holding u = q + 8 of elements k = 8w .. 8w+7: bits 4i..4i+3 hold element 8w + 2i and bits
+16+4i..16+4i+3 hold element 8w + 2i + 1, for i = 0..3 (even elements in the low half-word, odd
+elements in the high half-word, each in k order).  One 16-byte run of four words is exactly one
+group of 32.  Scales[r, g] is the bf16 scale of elements 32g..32g+31 of row r.
 """
 from __future__ import annotations
 
@@ -45,8 +46,13 @@ REPRODUCE_TOL = 1.0 / 16.0
 # packed layout
 # ------------------------------------------------------------------------------------------
 
+def nibble_shift(j: int) -> int:
+    """Bit offset of element 8w + j inside word w: even j in the low half-word, odd j in the high."""
+    return 4 * (j // 2) + (16 if j % 2 else 0)
+
+
 def pack(q) -> np.ndarray:
-    """int codes [R, K] in -8..7 -> uint32 words [R, K/8] (nibble j of word w = element 8w+j)."""
+    """int codes [R, K] in -8..7 -> uint32 words [R, K/8] in the layout described above."""
     q = np.asarray(q, dtype=np.int64)
     R, K = q.shape
     assert K % 8 == 0
@@ -54,7 +60,7 @@ def pack(q) -> np.ndarray:
     u = (q + 8).astype(np.uint64).reshape(R, K // 8, 8)
     word = np.zeros((R, K // 8), dtype=np.uint64)
     for j in range(8):
-        word |= u[:, :, j] << np.uint64(4 * j)
+        word |= u[:, :, j] << np.uint64(nibble_shift(j))
     return word.astype(np.uint32)
 
 
@@ -64,7 +70,7 @@ def unpack(codes) -> np.ndarray:
     R, W = c.shape
     q = np.empty((R, W, 8), dtype=np.int64)
     for j in range(8):
-        q[:, :, j] = ((c >> np.uint64(4 * j)) & np.uint64(0xF)).astype(np.int64) - 8
+        q[:, :, j] = ((c >> np.uint64(nibble_shift(j))) & np.uint64(0xF)).astype(np.int64) - 8
     return q.reshape(R, W * 8)
 
 

@@ -157,7 +157,8 @@ __global__ void __launch_bounds__(256) repack_kernel(const uint4* __restrict__ w
     for (int wd = 0; wd < 4; ++wd) {
       uint32_t word = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) word |= static_cast<uint32_t>(q[8 * wd + j] + 8) << (4 * j);
+      for (int j = 0; j < 8; ++j)   // even elements in the low half-word, odd in the high
+        word |= static_cast<uint32_t>(q[8 * wd + j] + 8) << (4 * (j >> 1) + 16 * (j & 1));
       pw[wd] = word;
     }
     codes[gi] = packed;

@@ -9,41 +9,49 @@
 // "1. Why quantization pays off").
 //
 // Design (sm_100a):
-//   * Work unit = (expert e, token block of <= 32 routed rows, tile of 128 weight rows, K split).
-//     A persistent grid (one CTA per SM) walks the units; the unit table is a prefix sum over
+//   * Work unit = (expert e, block of <= 16 routed rows, tile of 128 weight rows, K split).  A
+//     persistent grid (two CTAs per SM) walks the units; the unit table is a prefix sum over the
 //     experts built on the device from expert_offsets, so no host synchronisation is needed.
-//   * One producer warp feeds a 4-stage shared-memory ring: per stage 8 groups (256 k) of the
-//     128-row code tile by a 2-D TMA copy with the 128-byte swizzle (two 64-row boxes), the
-//     matching bf16 scales by 4-byte cp.async, and the <= 32 activation rows (gathered by
-//     a_row_of_pair) by 1-D bulk copies, all completing on one mbarrier.
-//   * Eight consumer warps each own 16 weight rows.  A thread's 32-bit code word is turned into
-//     four bf16 pairs (one lop3 + one packed fma per pair), which are exactly the A fragments of
-//     two m16n8k16 MMAs, with the tokens as the n = 8 side.  The MMA's k order is permuted so
-//     that word t of a group feeds quad position t; the activation pairs are permuted to match
-//     with prmt.  Each group's two MMAs start from zero and the group's bf16 scale is folded in
-//     with one fp32 FMA per accumulator: acc += s_g * (sum over the group of q * x).  Products
-//     q * x are exact in fp32.
-//   * Epilogue through shared memory: bf16 rows, the GELU gate (gate rows in warps 0-3, up rows
-//     in warps 4-7 of the same tile), or float32 split-K partials reduced in a fixed order by
-//     the last CTA of the tile (deterministic).
+//   * A 3-stage shared-memory ring per CTA (6 stages in flight per SM).  One stage = 8 groups
+//     (256 k) of the 128-row code tile (two 64-row 2-D TMA boxes, 128-byte swizzle), the matching
+//     bf16 scales (two 2-D TMA boxes when the scale row pitch is 16-byte aligned, else the tile's
+//     contiguous 64-row scale blocks by 1-D bulk copy), and the <= 16 activation rows gathered by
+//     a_row_of_pair (1-D bulk copies).  Everything completes on the stage's mbarrier.  Lane 0 of
+//     warp 0 issues the copies one ring-length ahead of the math.
+//   * Eight warps each own 16 weight rows.  A thread's 32-bit code word becomes four bf16 pairs
+//     (one lop3 + one packed fma per pair), which are exactly the A fragments of two m16n8k16
+//     MMAs with the tokens as the n = 8 side.  The packed nibble order puts two consecutive k in
+//     each extracted pair, so the activation B fragments are plain 16-byte shared loads.  Each
+//     group's MMAs start from zero and the group's scale is folded in with one fp32 FMA per
+//     accumulator: acc += s_g * (sum over the group of q * x).  Products q * x are exact in fp32.
+//   * Epilogue from registers, without a CTA barrier: with the GELU gate each warp's two A-fragment
+//     row sets are 8 gate rows and the 8 up rows of the same outputs, so h = gelu(g) * u is formed
+//     in the thread that holds both.  Dense split-K writes float32 partials that the last CTA of
+//     the tile reduces in a fixed order (deterministic).
 #include <cudaTypedefs.h>
+
+#include <cstring>
 
 #include "common.cuh"
 
 namespace w4 {
 
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kGS = 8;                        // groups per stage
-constexpr int kCWarps = 8;                    // consumer warps
-constexpr int kBN = 16 * kCWarps;             // weight rows per tile
+constexpr int kWarps = 8;                     // all warps compute; warp 0 also issues the copies
+constexpr int kThreads = kWarps * 32;
+constexpr int kBN = 16 * kWarps;              // weight rows per tile
 constexpr int kHalf = kBN / 2;                // rows per TMA box
-constexpr int kMT = 32;                       // routed rows (tokens) per unit
+constexpr int kMT = 16;                       // routed rows (tokens) per unit
 constexpr int kXPitch = kGS * 64 + 64;        // bytes per token row in an activation stage
 constexpr int kCodeBytes = kBN * kGS * 16;    // 16 KB
-constexpr int kXBytes = kMT * kXPitch;        // 18 KB
-constexpr int kScaleBytes = kBN * kGS * 2;    // 2 KB
+constexpr int kXBytes = kMT * kXPitch;        // 9 KB
+constexpr int kBlockMaxKg = 24;               // scale-block mode: two 64-row blocks of <= 24 groups
+constexpr int kScaleBytes = 2 * kHalf * kBlockMaxKg * 2;   // 6 KB
 constexpr int kEpPitch = kBN + 4;             // floats per token row in the epilogue buffer
-constexpr int kThreads = (kCWarps + 1) * 32;
+constexpr int kCtasPerSm = 2;
+
+enum ScaleMode { kScaleLdg = 0, kScaleBlock = 1, kScaleTma = 2 };
 
 struct StreamArgs {
   const uint16_t* a;
@@ -59,7 +67,7 @@ struct StreamArgs {
   float* partial;           // [splits, rows, N] (splits > 1)
   int32_t* counters;        // [tiles] (splits > 1)
   int splits, stages_per_split, n_tiles;
-  int scale_mode;           // 1: producer cp.async (kg even); 0: consumers load from global
+  int scale_mode;
   int32_t* dev_status;
 };
 
@@ -120,16 +128,6 @@ __device__ __forceinline__ bool tile_row_valid(const StreamArgs& A, const Unit& 
   return U.nt * kBN + r < A.N;
 }
 
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"r"(kCWarps * 32) : "memory");
-}
-
 // Source row in `a` of routed row r (checked; out-of-range indices read row 0 and are reported).
 __device__ __forceinline__ int64_t gather_row(const StreamArgs& A, int64_t r) {
   int64_t src = A.a_row_of_pair ? static_cast<int64_t>(__ldg(A.a_row_of_pair + r) / A.k_div) : r;
@@ -140,8 +138,79 @@ __device__ __forceinline__ int64_t gather_row(const StreamArgs& A, int64_t r) {
   return src;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes, StreamArgs A) {
+// The copy side of the ring: a cursor over (unit, stage) that runs kStages - 1 stages ahead.
+struct Producer {
+  int64_t u;
+  Unit U;
+  int g;
+  int64_t src_row;
+  bool done;
+};
+
+__device__ __forceinline__ void producer_load_unit(const StreamArgs& A, const int* table, const int* offs,
+                                                   int64_t total, Producer& P, int lane) {
+  P.done = P.u >= total;
+  if (P.done) return;
+  decode_unit(A, table, offs, P.u, P.U);
+  P.g = P.U.g0;
+  P.src_row = lane < P.U.mt ? gather_row(A, P.U.r0 + lane) : 0;
+}
+
+// Issues the stage under the cursor into its ring slot (warp-wide call) and advances the
+// cursor.  Returns false if the bounded wait for the slot gave up.
+__device__ __forceinline__ bool producer_issue(const StreamArgs& A, const CUtensorMap* tm_codes,
+                                               const CUtensorMap* tm_scales, uint8_t* smem,
+                                               uint64_t* full, uint64_t* empty, const int* table,
+                                               const int* offs, int64_t total, Producer& P,
+                                               uint32_t stage_index, int lane) {
+  if (P.done) return true;
+  const int slot = stage_index % kStages;
+  const uint32_t round = stage_index / kStages;
+  if (round > 0) {
+    bool ok = true;
+    if (lane == 0) ok = mbar_wait(&empty[slot], (round - 1) & 1);
+    if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+  }
+  const Unit& U = P.U;
+  const int g = P.g;
+  const int gc = min(kGS, U.g1 - g);
+  uint8_t* cdst = smem + SmemLayout::codes + slot * kCodeBytes;
+  uint8_t* xdst = smem + SmemLayout::x + slot * kXBytes;
+  uint8_t* sdst = smem + SmemLayout::sc + slot * kScaleBytes;
+  const uint32_t xbytes = static_cast<uint32_t>(gc) * 64u;
+  if (lane == 0) {
+    const int64_t row_a = tile_row(A, U, 0);
+    const int64_t row_b = tile_row(A, U, kHalf);
+    uint32_t sbytes = 0;
+    if (A.scale_mode == kScaleTma) sbytes = 2 * kHalf * kGS * 2;
+    else if (A.scale_mode == kScaleBlock) sbytes = 2 * kHalf * A.kg * 2;
+    mbar_arrive_expect_tx(&full[slot], kCodeBytes + sbytes + xbytes * U.mt);
+    tma_load_2d(cdst, tm_codes, g * 4, static_cast<int32_t>(row_a), &full[slot]);
+    tma_load_2d(cdst + kHalf * 128, tm_codes, g * 4, static_cast<int32_t>(row_b), &full[slot]);
+    if (A.scale_mode == kScaleTma) {
+      tma_load_2d(sdst, tm_scales, g, static_cast<int32_t>(row_a), &full[slot]);
+      tma_load_2d(sdst + kHalf * kGS * 2, tm_scales, g, static_cast<int32_t>(row_b), &full[slot]);
+    } else if (A.scale_mode == kScaleBlock) {
+      const uint32_t blk = kHalf * A.kg * 2;
+      bulk_g2s(sdst, A.scales + row_a * A.kg, blk, &full[slot]);
+      bulk_g2s(sdst + blk, A.scales + row_b * A.kg, blk, &full[slot]);
+    }
+  }
+  __syncwarp();
+  if (lane < U.mt)
+    bulk_g2s(xdst + lane * kXPitch, A.a + P.src_row * A.K + static_cast<int64_t>(g) * 32, xbytes,
+             &full[slot]);
+  P.g += kGS;
+  if (P.g >= U.g1) {
+    P.u += gridDim.x;
+    producer_load_unit(A, table, offs, total, P, lane);
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
+                   const __grid_constant__ CUtensorMap tmap_scales, StreamArgs A) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + SmemLayout::bars);
@@ -190,8 +259,8 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes, StreamArgs A)
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1 + (A.scale_mode ? 32 : 0));
-      mbar_init(&empty[s], kCWarps);
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kWarps);
     }
     flags[0] = 0;
     fence_barrier_init();
@@ -199,74 +268,29 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes, StreamArgs A)
   __syncthreads();
   const int64_t total_units = table[A.E];
 
-  if (warp == kCWarps) {
-    // ------------------------------- producer -------------------------------
-    if (lane == 0) prefetch_tmap(&tmap_codes);
-    uint32_t it = 0;
-    int64_t u = blockIdx.x;
-    Unit U;
-    int64_t src_row = 0;
-    if (u < total_units) {
-      decode_unit(A, table, offs, u, U);
-      if (lane < U.mt) src_row = gather_row(A, U.r0 + lane);
+  Producer P;
+  uint32_t issued = 0;
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tmap_codes);
+      if (A.scale_mode == kScaleTma) prefetch_tmap(&tmap_scales);
     }
-    while (u < total_units) {
-      // prefetch the next unit's gather rows while this unit's stages are issued
-      const int64_t un = u + gridDim.x;
-      Unit Un;
-      int64_t src_next = 0;
-      if (un < total_units) {
-        decode_unit(A, table, offs, un, Un);
-        if (lane < Un.mt) src_next = gather_row(A, Un.r0 + lane);
-      }
-      const int64_t row_a = tile_row(A, U, 0);
-      const int64_t row_b = tile_row(A, U, kHalf);
-      for (int g = U.g0; g < U.g1; g += kGS, ++it) {
-        const int slot = it % kStages;
-        const uint32_t round = it / kStages;
-        const int gc = min(kGS, U.g1 - g);
-        if (round > 0) {
-          bool ok = true;
-          if (lane == 0) ok = mbar_wait(&empty[slot], (round - 1) & 1);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (!ok || flags[0]) {
-            if (lane == 0) { set_status(A.dev_status, W4_ERR_TIMEOUT); flags[0] = 1; }
-            return;
-          }
-        }
-        uint8_t* cdst = smem + SmemLayout::codes + slot * kCodeBytes;
-        uint8_t* xdst = smem + SmemLayout::x + slot * kXBytes;
-        const uint32_t xbytes = static_cast<uint32_t>(gc) * 64u;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full[slot], kCodeBytes + xbytes * U.mt);
-          tma_load_2d(cdst, &tmap_codes, g * 4, static_cast<int32_t>(row_a), &full[slot]);
-          tma_load_2d(cdst + kHalf * 128, &tmap_codes, g * 4, static_cast<int32_t>(row_b), &full[slot]);
-        }
-        __syncwarp();
-        if (lane < U.mt)
-          bulk_g2s(xdst + lane * kXPitch, A.a + src_row * A.K + static_cast<int64_t>(g) * 32, xbytes,
-                   &full[slot]);
-        if (A.scale_mode) {
-          const uint32_t sdst = smem_u32(smem + SmemLayout::sc + slot * kScaleBytes);
-#pragma unroll 1
-          for (int r = lane; r < kBN; r += 32) {
-            const int64_t grow = tile_row_valid(A, U, r) ? tile_row(A, U, r) : row_a;
-            const uint16_t* src = A.scales + grow * A.kg + g;
-            for (int p = 0; p < gc; p += 2) cp_async4(sdst + r * 16 + p * 2, src + p);
-          }
-          cp_async_arrive_noinc(&full[slot]);
-        }
-      }
-      u = un;
-      U = Un;
-      src_row = src_next;
-    }
-    return;
+    P.u = blockIdx.x;
+    producer_load_unit(A, table, offs, total_units, P, lane);
+    for (; issued < kStages - 1 && !P.done; ++issued)
+      producer_issue(A, &tmap_codes, &tmap_scales, smem, full, empty, table, offs, total_units, P,
+                     issued, lane);
   }
 
-  // ------------------------------- consumers -------------------------------
+  // Rows of this thread's two A-fragment rows.  GELU gate: rlo = gate row j, rhi = up row j of
+  // the same j (tile rows 8w+gid and 64+8w+gid), so the gate is applied in registers.  Otherwise
+  // 16 consecutive rows per warp.
   const int gid = lane >> 2, tq = lane & 3;
-  const int rlo = warp * 16 + gid, rhi = rlo + 8;
+  const bool gelu = (A.epi == W4_EPI_GELU_GATE);
+  const int rlo = gelu ? warp * 8 + gid : warp * 16 + gid;
+  const int rhi = gelu ? rlo + kHalf : rlo + 8;
+  const int r7 = rlo & 7;                       // == rhi & 7
+  const int dw = (rhi - rlo) * 32;              // word distance between the two rows
   float* ep = reinterpret_cast<float*>(smem + SmemLayout::ep);
   uint32_t it = 0;
   bool aborted = false;   // after a timed-out wait: skip work, keep every barrier
@@ -274,15 +298,22 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes, StreamArgs A)
     Unit U;
     decode_unit(A, table, offs, u, U);
     const int nblk = (U.mt + 7) >> 3;
-    float acc[4][4];
+    float acc[2][4];
 #pragma unroll
-    for (int b = 0; b < 4; ++b)
+    for (int b = 0; b < 2; ++b)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[b][i] = 0.f;
-    const int64_t grow_lo = tile_row_valid(A, U, rlo) ? tile_row(A, U, rlo) : tile_row(A, U, 0);
-    const int64_t grow_hi = tile_row_valid(A, U, rhi) ? tile_row(A, U, rhi) : tile_row(A, U, 0);
 
     for (int g = U.g0; g < U.g1; g += kGS, ++it) {
+      // keep the ring full: warp 0 issues the stage kStages - 1 ahead of this one
+      if (warp == 0 && !aborted && !P.done) {
+        if (!producer_issue(A, &tmap_codes, &tmap_scales, smem, full, empty, table, offs,
+                            total_units, P, issued, lane)) {
+          if (lane == 0) { set_status(A.dev_status, W4_ERR_TIMEOUT); flags[0] = 1; }
+          aborted = true;
+        }
+        ++issued;
+      }
       const int slot = it % kStages;
       const uint32_t round = it / kStages;
       const int gc = min(kGS, U.g1 - g);
@@ -293,13 +324,26 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes, StreamArgs A)
       if (aborted) continue;
       const uint32_t* cw = reinterpret_cast<const uint32_t*>(smem + SmemLayout::codes + slot * kCodeBytes);
       const uint8_t* xs = smem + SmemLayout::x + slot * kXBytes;
+      const uint8_t* ss = smem + SmemLayout::sc + slot * kScaleBytes;
+      // scales of rows rlo / rhi for the stage's 8 groups, two bf16 per word
       uint32_t slo[4], shi[4];
-      if (A.scale_mode) {
-        const uint4* sc = reinterpret_cast<const uint4*>(smem + SmemLayout::sc + slot * kScaleBytes);
-        const uint4 vlo = sc[rlo], vhi = sc[rhi];
+      if (A.scale_mode == kScaleTma) {
+        const uint4 vlo = *reinterpret_cast<const uint4*>(ss + rlo * 16);
+        const uint4 vhi = *reinterpret_cast<const uint4*>(ss + rhi * 16);
         slo[0] = vlo.x; slo[1] = vlo.y; slo[2] = vlo.z; slo[3] = vlo.w;
         shi[0] = vhi.x; shi[1] = vhi.y; shi[2] = vhi.z; shi[3] = vhi.w;
+      } else if (A.scale_mode == kScaleBlock) {
+        // block rows hold all kg groups (kg even, g a multiple of 8: 4-byte aligned pairs)
+        const uint32_t* plo = reinterpret_cast<const uint32_t*>(ss + (rlo * A.kg + g) * 2);
+        const uint32_t* phi = reinterpret_cast<const uint32_t*>(ss + (rhi * A.kg + g) * 2);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          slo[p] = 2 * p < gc ? plo[p] : 0u;
+          shi[p] = 2 * p < gc ? phi[p] : 0u;
+        }
       } else {
+        const int64_t grow_lo = tile_row_valid(A, U, rlo) ? tile_row(A, U, rlo) : tile_row(A, U, 0);
+        const int64_t grow_hi = tile_row_valid(A, U, rhi) ? tile_row(A, U, rhi) : tile_row(A, U, 0);
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
           const int ga = g + 2 * p, gb = g + 2 * p + 1;
@@ -311,46 +355,55 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes, StreamArgs A)
           shi[p] = h0 | (h1 << 16);
         }
       }
-      // Dequantise the stage's 8 groups for rows rlo / rhi into MMA A fragments.  The word of
-      // row r, group gi, quad position tq sits at chunk (gi ^ r%8) of the row (128-byte swizzle).
-      uint32_t fa[kGS][8];
-      float fsl[kGS], fsh[kGS];
+      // Two halves of 4 groups: dequantise rows rlo / rhi into MMA A fragments, then run the
+      // token blocks.  Word (row r, group gi, quad position tq) sits at chunk gi ^ (r % 8) of the
+      // 128-byte row (TMA 128-byte swizzle).  Each extracted bf16 pair is two consecutive k, so
+      // k-step 0 takes elements 8tq+0..3 (x pairs .x, .y) and k-step 1 elements 8tq+4..7 (.z, .w).
+      // rows rlo and rhi share the swizzle phase (rlo % 8): one address per group
+      const uint32_t* cwl = cw + rlo * 32 + tq;
+      const bool mask_tail = (A.scale_mode != kScaleTma) && gc < kGS;   // TMA zero-fills past K
 #pragma unroll
-      for (int gi = 0; gi < kGS; ++gi) {
-        const uint32_t wlo = cw[rlo * 32 + ((gi ^ (rlo & 7)) << 2) + tq];
-        const uint32_t whi = cw[rhi * 32 + ((gi ^ (rhi & 7)) << 2) + tq];
-        fa[gi][0] = nibbles_to_bf16x2(wlo);        // k-step 0: nibbles (0,4) | (1,5)
-        fa[gi][1] = nibbles_to_bf16x2(whi);
-        fa[gi][2] = nibbles_to_bf16x2(wlo >> 4);
-        fa[gi][3] = nibbles_to_bf16x2(whi >> 4);
-        fa[gi][4] = nibbles_to_bf16x2(wlo >> 8);   // k-step 1: nibbles (2,6) | (3,7)
-        fa[gi][5] = nibbles_to_bf16x2(whi >> 8);
-        fa[gi][6] = nibbles_to_bf16x2(wlo >> 12);
-        fa[gi][7] = nibbles_to_bf16x2(whi >> 12);
-        const uint32_t sl = (gi & 1) ? (slo[gi >> 1] & 0xFFFF0000u) : (slo[gi >> 1] << 16);
-        const uint32_t sh = (gi & 1) ? (shi[gi >> 1] & 0xFFFF0000u) : (shi[gi >> 1] << 16);
-        fsl[gi] = gi < gc ? __uint_as_float(sl) : 0.f;   // groups past the K range add nothing
-        fsh[gi] = gi < gc ? __uint_as_float(sh) : 0.f;
-      }
+      for (int h = 0; h < kGS; h += 4) {
+        uint32_t fa[4][8];
+        float fsl[4], fsh[4];
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        if (b < nblk) {
-          const uint8_t* xrow = xs + (b * 8 + gid) * kXPitch + tq * 16;
+        for (int i = 0; i < 4; ++i) {
+          const int gi = h + i;
+          const uint32_t* pw = cwl + ((gi ^ r7) << 2);
+          const uint32_t wlo = pw[0];
+          const uint32_t whi = pw[dw];
+          fa[i][0] = nibbles_to_bf16x2(wlo);        // k-step 0: elements (0,1) | (2,3)
+          fa[i][1] = nibbles_to_bf16x2(whi);
+          fa[i][2] = nibbles_to_bf16x2(wlo >> 4);
+          fa[i][3] = nibbles_to_bf16x2(whi >> 4);
+          fa[i][4] = nibbles_to_bf16x2(wlo >> 8);   // k-step 1: elements (4,5) | (6,7)
+          fa[i][5] = nibbles_to_bf16x2(whi >> 8);
+          fa[i][6] = nibbles_to_bf16x2(wlo >> 12);
+          fa[i][7] = nibbles_to_bf16x2(whi >> 12);
+          const uint32_t sl = (gi & 1) ? (slo[gi >> 1] & 0xFFFF0000u) : (slo[gi >> 1] << 16);
+          const uint32_t sh = (gi & 1) ? (shi[gi >> 1] & 0xFFFF0000u) : (shi[gi >> 1] << 16);
+          fsl[i] = __uint_as_float(sl);
+          fsh[i] = __uint_as_float(sh);
+          if (mask_tail && gi >= gc) { fsl[i] = 0.f; fsh[i] = 0.f; }   // past the K range
+        }
 #pragma unroll
-          for (int gi = 0; gi < kGS; ++gi) {
-            const uint4 xv = *reinterpret_cast<const uint4*>(xrow + gi * 64);
-            const uint32_t b00 = prmt(xv.x, xv.z, 0x5410), b01 = prmt(xv.x, xv.z, 0x7632);
-            const uint32_t b10 = prmt(xv.y, xv.w, 0x5410), b11 = prmt(xv.y, xv.w, 0x7632);
-            const uint32_t a0[4] = {fa[gi][0], fa[gi][1], fa[gi][2], fa[gi][3]};
-            const uint32_t a1[4] = {fa[gi][4], fa[gi][5], fa[gi][6], fa[gi][7]};
-            float d[4];
-            const float z[4] = {0.f, 0.f, 0.f, 0.f};
-            mma_bf16_16816(d, a0, b00, b01, z);
-            mma_bf16_16816(d, a1, b10, b11, d);
-            acc[b][0] = fmaf(fsl[gi], d[0], acc[b][0]);
-            acc[b][1] = fmaf(fsl[gi], d[1], acc[b][1]);
-            acc[b][2] = fmaf(fsh[gi], d[2], acc[b][2]);
-            acc[b][3] = fmaf(fsh[gi], d[3], acc[b][3]);
+        for (int b = 0; b < 2; ++b) {
+          if (b < nblk) {
+            const uint8_t* xrow = xs + (b * 8 + gid) * kXPitch + tq * 16;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 xv = *reinterpret_cast<const uint4*>(xrow + (h + i) * 64);
+              const uint32_t a0[4] = {fa[i][0], fa[i][1], fa[i][2], fa[i][3]};
+              const uint32_t a1[4] = {fa[i][4], fa[i][5], fa[i][6], fa[i][7]};
+              float d[4];
+              const float z[4] = {0.f, 0.f, 0.f, 0.f};
+              mma_bf16_16816(d, a0, xv.x, xv.y, z);
+              mma_bf16_16816(d, a1, xv.z, xv.w, d);
+              acc[b][0] = fmaf(fsl[i], d[0], acc[b][0]);
+              acc[b][1] = fmaf(fsl[i], d[1], acc[b][1]);
+              acc[b][2] = fmaf(fsh[i], d[2], acc[b][2]);
+              acc[b][3] = fmaf(fsh[i], d[3], acc[b][3]);
+            }
           }
         }
       }
@@ -359,8 +412,42 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes, StreamArgs A)
     }
 
     // --------------------------- epilogue ---------------------------
+    if (A.splits == 1) {
+      // straight from registers: thread holds rows rlo / rhi for tokens 2tq, 2tq + 1 of each block
+      if (!aborted) {
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
+        for (int b = 0; b < 2; ++b) {
+          if (b < nblk) {
+            const int t0 = b * 8 + 2 * tq;
+            if (gelu) {
+              const int Nh = A.N >> 1;
+              const int j = U.nt * kHalf + warp * 8 + gid;
+              if (j < Nh) {
+                if (t0 < U.mt)
+                  A.out[(U.r0 + t0) * Nh + j] = f32_to_bf16_bits(gelu_tanh(acc[b][0]) * acc[b][2]);
+                if (t0 + 1 < U.mt)
+                  A.out[(U.r0 + t0 + 1) * Nh + j] = f32_to_bf16_bits(gelu_tanh(acc[b][1]) * acc[b][3]);
+              }
+            } else {
+              const int nlo = U.nt * kBN + rlo, nhi = nlo + 8;
+              if (t0 < U.mt) {
+                if (nlo < A.N) A.out[(U.r0 + t0) * A.N + nlo] = f32_to_bf16_bits(acc[b][0]);
+                if (nhi < A.N) A.out[(U.r0 + t0) * A.N + nhi] = f32_to_bf16_bits(acc[b][2]);
+              }
+              if (t0 + 1 < U.mt) {
+                if (nlo < A.N) A.out[(U.r0 + t0 + 1) * A.N + nlo] = f32_to_bf16_bits(acc[b][1]);
+                if (nhi < A.N) A.out[(U.r0 + t0 + 1) * A.N + nhi] = f32_to_bf16_bits(acc[b][3]);
+              }
+            }
+          }
+        }
+      }
+      continue;
+    }
+    // split-K (dense, no gate): float32 partials through shared memory, then the last CTA of the
+    // tile reduces them in split order
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
       if (b < nblk) {
         const int t0 = b * 8 + 2 * tq;
         ep[t0 * kEpPitch + rlo] = acc[b][0];
@@ -369,78 +456,42 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes, StreamArgs A)
         ep[(t0 + 1) * kEpPitch + rhi] = acc[b][3];
       }
     }
-    consumer_sync();
-    const int ctid = threadIdx.x;  // 0..255
-    if (flags[0]) {
-      // aborted CTA: write nothing, keep the barrier count of the normal path
-      if (A.epi != W4_EPI_GELU_GATE && A.splits > 1) { consumer_sync(); consumer_sync(); }
-    } else if (A.epi == W4_EPI_GELU_GATE) {
-      const int Nh = A.N >> 1;
-      const int j0 = U.nt * kHalf;
-      for (int idx = ctid; idx < U.mt * (kHalf / 8); idx += kCWarps * 32) {
-        const int t = idx / (kHalf / 8), c = idx % (kHalf / 8);
-        const float* gp = ep + t * kEpPitch + c * 8;
-        const float* up = gp + kHalf;
-        float h[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) h[i] = gelu_tanh(gp[i]) * up[i];
-        uint16_t* dst = A.out + (U.r0 + t) * Nh + j0 + c * 8;
-        if (j0 + c * 8 + 8 <= Nh && (Nh & 7) == 0) {
-          uint4 v;
-          v.x = pack_bf16x2(h[0], h[1]); v.y = pack_bf16x2(h[2], h[3]);
-          v.z = pack_bf16x2(h[4], h[5]); v.w = pack_bf16x2(h[6], h[7]);
-          *reinterpret_cast<uint4*>(dst) = v;
-        } else {
-          for (int i = 0; i < 8 && j0 + c * 8 + i < Nh; ++i) dst[i] = f32_to_bf16_bits(h[i]);
-        }
-      }
-    } else if (A.splits == 1) {
-      const int n0 = U.nt * kBN;
-      for (int idx = ctid; idx < U.mt * (kBN / 8); idx += kCWarps * 32) {
-        const int t = idx / (kBN / 8), c = idx % (kBN / 8);
-        const float* src = ep + t * kEpPitch + c * 8;
-        uint16_t* dst = A.out + (U.r0 + t) * A.N + n0 + c * 8;
-        if (n0 + c * 8 + 8 <= A.N && (A.N & 7) == 0) {
-          uint4 v;
-          v.x = pack_bf16x2(src[0], src[1]); v.y = pack_bf16x2(src[2], src[3]);
-          v.z = pack_bf16x2(src[4], src[5]); v.w = pack_bf16x2(src[6], src[7]);
-          *reinterpret_cast<uint4*>(dst) = v;
-        } else {
-          for (int i = 0; i < 8 && n0 + c * 8 + i < A.N; ++i) dst[i] = f32_to_bf16_bits(src[i]);
-        }
-      }
-    } else {
-      // split-K: float32 partial, then the last CTA of the tile reduces in split order
-      const int n0 = U.nt * kBN;
-      for (int idx = ctid; idx < U.mt * kBN; idx += kCWarps * 32) {
+    __syncthreads();
+    const int ctid = threadIdx.x;
+    const int n0 = U.nt * kBN;
+    if (!flags[0]) {
+      for (int idx = ctid; idx < U.mt * kBN; idx += kThreads) {
         const int t = idx / kBN, c = idx % kBN;
         if (n0 + c < A.N)
           A.partial[(static_cast<int64_t>(U.sp) * A.rows + U.r0 + t) * A.N + n0 + c] = ep[t * kEpPitch + c];
       }
-      __threadfence();
-      consumer_sync();
-      if (ctid == 0) {
+    }
+    __threadfence();
+    __syncthreads();
+    if (ctid == 0) {
+      int last = 0;
+      if (!flags[0]) {
         const int tile = U.tb * A.n_tiles + U.nt;
         const int prev = atomicAdd(&A.counters[tile], 1);
-        const int last = (prev == A.splits - 1);
+        last = (prev == A.splits - 1);
         if (last) A.counters[tile] = 0;
-        flags[1] = last;
       }
-      consumer_sync();
-      if (flags[1]) {
-        __threadfence();
-        for (int idx = ctid; idx < U.mt * kBN; idx += kCWarps * 32) {
-          const int t = idx / kBN, c = idx % kBN;
-          if (n0 + c < A.N) {
-            float s = 0.f;
-            for (int sp = 0; sp < A.splits; ++sp)
-              s += __ldcg(&A.partial[(static_cast<int64_t>(sp) * A.rows + U.r0 + t) * A.N + n0 + c]);
-            A.out[(U.r0 + t) * A.N + n0 + c] = f32_to_bf16_bits(s);
-          }
+      flags[1] = last;
+    }
+    __syncthreads();
+    if (flags[1]) {
+      __threadfence();
+      for (int idx = ctid; idx < U.mt * kBN; idx += kThreads) {
+        const int t = idx / kBN, c = idx % kBN;
+        if (n0 + c < A.N) {
+          float sum = 0.f;
+          for (int sp = 0; sp < A.splits; ++sp)
+            sum += __ldcg(&A.partial[(static_cast<int64_t>(sp) * A.rows + U.r0 + t) * A.N + n0 + c]);
+          A.out[(U.r0 + t) * A.N + n0 + c] = f32_to_bf16_bits(sum);
         }
       }
     }
-    consumer_sync();
+    __syncthreads();
   }
 }
 
@@ -476,6 +527,20 @@ static bool encode_codes_map(CUtensorMap* m, const uint32_t* codes, int64_t rows
   return r == CUDA_SUCCESS;
 }
 
+// Scales [rows_total, kg] bf16 as a 2-D tensor (kg % 8 == 0): box = 8 groups x 64 rows.
+static bool encode_scales_map(CUtensorMap* m, const uint16_t* scales, int64_t rows_total, int kg) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kg), static_cast<cuuint64_t>(rows_total)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kg) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(w4::kGS), static_cast<cuuint32_t>(w4::kHalf)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t*>(scales), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 static size_t stream_smem_bytes(int E) {
   return w4::SmemLayout::bytes_without_table + static_cast<size_t>(E + 1) * 8 + 1024;
 }
@@ -492,11 +557,11 @@ static StreamPlan plan_stream(int64_t rows, int N, int K, int E, int epi, bool d
                                         : (N + w4::kBN - 1) / w4::kBN;
   p.splits = 1;
   if (dense) {
-    // split K while the units do not fill the SMs four times over and the float32 partials stay
-    // below ~1/8 of the weight bytes
+    // split K while the units do not fill the CTAs four times over and the float32 partials
+    // stay below ~1/8 of the weight bytes
     const int64_t ntb = (rows + w4::kMT - 1) / w4::kMT;
     const double wbytes = static_cast<double>(N) * K * 0.5625;
-    while (p.splits * 2 <= kstages && ntb * p.n_tiles * p.splits < 4LL * sm_count &&
+    while (p.splits * 2 <= kstages && ntb * p.n_tiles * p.splits < 4LL * w4::kCtasPerSm * sm_count &&
            static_cast<double>(p.splits * 2) * rows * N * 8.0 <= wbytes / 8.0)
       p.splits *= 2;
   }
@@ -527,8 +592,20 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
   A.E = E; A.N = N; A.K = K; A.kg = K / 32; A.rows = rows; A.epi = epi; A.out = out;
   A.a_rows = a_row_of_pair ? rows / A.k_div : rows;
   A.splits = p.splits; A.stages_per_split = p.stages_per_split; A.n_tiles = p.n_tiles;
-  A.scale_mode = (A.kg % 2 == 0) ? 1 : 0;
   A.dev_status = dev_status;
+  // Scale staging: 2-D TMA when a scale row is a whole number of 16-byte chunks; else the tile's
+  // contiguous 64-row scale blocks by bulk copy when they are 16-byte aligned and small; else
+  // direct loads.
+  const bool s16 = (reinterpret_cast<uintptr_t>(scales) & 15) == 0;
+  if (A.kg % 8 == 0 && s16) {
+    A.scale_mode = w4::kScaleTma;
+  } else if (p.splits == 1 && A.kg % 2 == 0 && A.kg <= w4::kBlockMaxKg && N % 8 == 0 && s16 &&
+             (epi == W4_EPI_GELU_GATE ? (N / 2) % w4::kHalf == 0 : N % w4::kBN == 0)) {
+    // (whole tiles only: the 64-row blocks are plain bulk copies and must stay inside the array)
+    A.scale_mode = w4::kScaleBlock;
+  } else {
+    A.scale_mode = w4::kScaleLdg;
+  }
   if (p.splits > 1) {
     const size_t need = w4_stream_workspace_bytes(rows, N, K, E, epi, dense, sm_count);
     if (ws == nullptr || ws_bytes < need) return W4_ERR_WORKSPACE;
@@ -538,8 +615,12 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
     A.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + pb);
   }
   if (rows == 0) return W4_OK;
-  CUtensorMap tmap;
+  CUtensorMap tmap, smap;
+  std::memset(&smap, 0, sizeof(smap));
   if (!encode_codes_map(&tmap, codes, static_cast<int64_t>(E) * N, K)) return W4_ERR_CUDA;
+  if (A.scale_mode == w4::kScaleTma &&
+      !encode_scales_map(&smap, scales, static_cast<int64_t>(E) * N, A.kg))
+    return W4_ERR_CUDA;
   const size_t smem = stream_smem_bytes(E);
   static int attr_done[64] = {0};
   int dev = 0;
@@ -548,8 +629,11 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
     if (cudaFuncSetAttribute(w4::stream_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(stream_smem_bytes(1024))) != cudaSuccess)
       return W4_ERR_CUDA;
+    if (cudaFuncSetAttribute(w4::stream_gemm_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+      return W4_ERR_CUDA;
     attr_done[dev] = 1;
   }
-  w4::stream_gemm_kernel<<<sm_count, w4::kThreads, smem, stream>>>(tmap, A);
+  w4::stream_gemm_kernel<<<sm_count * w4::kCtasPerSm, w4::kThreads, smem, stream>>>(tmap, smap, A);
   return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
