@@ -11,9 +11,12 @@ namespace w4 {
 
 constexpr int kGroup = 32;            // weights per scale along the input dimension
 
-// Iteration cap for every spin on an mbarrier.  try_wait already suspends the thread for a
-// hardware-defined window per call, so this bounds a wait to well under a second or two.
-constexpr uint32_t kSpinLimit = 1u << 22;
+// Every wait on an mbarrier gives up after this many nanoseconds of %globaltimer (then the
+// kernel reports W4_ERR_TIMEOUT instead of hanging).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Suspend-time hint for mbarrier.try_wait: a waiting thread sleeps up to this long (it wakes as
+// soon as the phase completes) instead of spinning.
+constexpr uint32_t kSuspendHintNs = 20000;
 
 // ------------------------------------------------------------------------------------------
 // scalar conversions
@@ -60,17 +63,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n .reg .pred p;\n"
-      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
       " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs) : "memory");
   return ok != 0;
 }
 
-// Bounded wait: returns false when the cap is hit (the caller reports W4_ERR_TIMEOUT).
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait: returns false once kWaitLimitNs have passed (the caller reports W4_ERR_TIMEOUT).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-  return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
 }
 
 // 1-D bulk copy global -> shared, completion counted in bytes on `bar`.
@@ -136,6 +148,16 @@ __device__ __forceinline__ uint32_t nibbles_to_bf16x2(uint32_t v) {
   asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(q) : "r"(r), "r"(0x3F803F80u), "r"(0xC308C308u));
   return q;
 }
+
+// Same fields, returned biased: the bf16 pair (128 + u), exact.  A caller that multiplies these
+// by x must subtract 136 * sum(x) (see kMinus136x2).
+__device__ __forceinline__ uint32_t nibbles_to_bf16x2_biased(uint32_t v) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(v), "r"(0x000F000Fu), "r"(0x43004300u));
+  return r;
+}
+
+constexpr uint32_t kMinus136x2 = 0xC308C308u;   // bf16 pair (-136, -136)
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;

@@ -9,21 +9,22 @@
 // "1. Why quantization pays off").
 //
 // Design (sm_100a):
-//   * Work unit = (expert e, block of <= 16 routed rows, tile of 128 weight rows, K split).  A
-//     persistent grid (two CTAs per SM) walks the units; the unit table is a prefix sum over the
-//     experts built on the device from expert_offsets, so no host synchronisation is needed.
-//   * A 3-stage shared-memory ring per CTA (6 stages in flight per SM).  One stage = 8 groups
+//   * Work unit = (expert e, block of <= MT routed rows (MT = 8 or 16), tile of 128 weight rows,
+//     K split).  A persistent grid (two CTAs per SM) walks the units; the unit table is a prefix
+//     sum over the experts built on the device from expert_offsets (no host synchronisation).
+//   * Each CTA = 8 compute warps + 1 producer warp.  The producer keeps a shared-memory ring as
+//     deep as the per-CTA shared-memory budget allows (4-6 stages) full: one stage = 8 groups
 //     (256 k) of the 128-row code tile (two 64-row 2-D TMA boxes, 128-byte swizzle), the matching
-//     bf16 scales (two 2-D TMA boxes when the scale row pitch is 16-byte aligned, else the tile's
-//     contiguous 64-row scale blocks by 1-D bulk copy), and the <= 16 activation rows gathered by
-//     a_row_of_pair (1-D bulk copies).  Everything completes on the stage's mbarrier.  Lane 0 of
-//     warp 0 issues the copies one ring-length ahead of the math.
-//   * Eight warps each own 16 weight rows.  A thread's 32-bit code word becomes four bf16 pairs
-//     (one lop3 + one packed fma per pair), which are exactly the A fragments of two m16n8k16
-//     MMAs with the tokens as the n = 8 side.  The packed nibble order puts two consecutive k in
-//     each extracted pair, so the activation B fragments are plain 16-byte shared loads.  Each
-//     group's MMAs start from zero and the group's scale is folded in with one fp32 FMA per
-//     accumulator: acc += s_g * (sum over the group of q * x).  Products q * x are exact in fp32.
+//     bf16 scales (two 2-D TMA boxes when a scale row is a whole number of 16-byte chunks, else the
+//     tile's contiguous 64-row scale blocks by 1-D bulk copy), and the activation rows gathered by
+//     a_row_of_pair (1-D bulk copies).  Everything completes on the stage's mbarrier.
+//   * A compute warp owns 16 weight rows.  A thread's 32-bit code word becomes four bf16 pairs
+//     128 + u (one lop3 per pair, exact), which are exactly the A fragments of two m16n8k16 MMAs
+//     with the tokens as the n = 8 side; two more MMAs with the constant A = -136 remove the bias
+//     (q = u - 8).  The packed nibble order puts two consecutive k in each extracted pair, so the
+//     activation B fragments are plain 16-byte shared loads.  Each group's MMAs start from zero
+//     and the group's scale is folded in with one fp32 FMA per accumulator:
+//     acc += s_g * (sum over the group of q * x).  Products q * x are exact in fp32.
 //   * Epilogue from registers, without a CTA barrier: with the GELU gate each warp's two A-fragment
 //     row sets are 8 gate rows and the 8 up rows of the same outputs, so h = gelu(g) * u is formed
 //     in the thread that holds both.  Dense split-K writes float32 partials that the last CTA of
@@ -36,22 +37,38 @@
 
 namespace w4 {
 
-constexpr int kStages = 3;
+#ifndef W4_STREAM_GROUPS_PER_PASS
+#define W4_STREAM_GROUPS_PER_PASS 2           // groups dequantised into registers at a time
+#endif
+
+constexpr int kMaxStages = 6;
 constexpr int kGS = 8;                        // groups per stage
-constexpr int kWarps = 8;                     // all warps compute; warp 0 also issues the copies
-constexpr int kThreads = kWarps * 32;
+constexpr int kGP = W4_STREAM_GROUPS_PER_PASS;
+constexpr int kWarps = 8;                     // compute warps
+constexpr int kThreads = (kWarps + 1) * 32;   // + one producer warp
 constexpr int kBN = 16 * kWarps;              // weight rows per tile
 constexpr int kHalf = kBN / 2;                // rows per TMA box
-constexpr int kMT = 16;                       // routed rows (tokens) per unit
 constexpr int kXPitch = kGS * 64 + 64;        // bytes per token row in an activation stage
 constexpr int kCodeBytes = kBN * kGS * 16;    // 16 KB
-constexpr int kXBytes = kMT * kXPitch;        // 9 KB
 constexpr int kBlockMaxKg = 24;               // scale-block mode: two 64-row blocks of <= 24 groups
-constexpr int kScaleBytes = 2 * kHalf * kBlockMaxKg * 2;   // 6 KB
 constexpr int kEpPitch = kBN + 4;             // floats per token row in the epilogue buffer
 constexpr int kCtasPerSm = 2;
+// shared memory one CTA may use when two share an SM (228 KB per SM, 1 KB reserved per CTA)
+constexpr int kSmemPerCta = (233472 - kCtasPerSm * 1024) / kCtasPerSm;
 
 enum ScaleMode { kScaleLdg = 0, kScaleBlock = 1, kScaleTma = 2 };
+
+// Shared-memory layout, fixed per launch (offsets from the 1024-byte aligned base).
+struct Layout {
+  int stages;
+  int x_off, x_bytes;        // activation ring: stages x (MT rows x kXPitch)
+  int sc_off, sc_bytes;      // scale ring: stages x sc_bytes
+  int ep_off;                // split-K epilogue buffer (MT x kEpPitch floats), or -1
+  int bar_off;               // 2 * stages mbarriers
+  int flag_off;              // 16 bytes
+  int table_off;             // int table[E + 1], int offs[E + 1]
+  int total;
+};
 
 struct StreamArgs {
   const uint16_t* a;
@@ -68,18 +85,8 @@ struct StreamArgs {
   int32_t* counters;        // [tiles] (splits > 1)
   int splits, stages_per_split, n_tiles;
   int scale_mode;
+  Layout L;
   int32_t* dev_status;
-};
-
-struct SmemLayout {
-  static constexpr int codes = 0;
-  static constexpr int x = codes + kStages * kCodeBytes;
-  static constexpr int sc = x + kStages * kXBytes;
-  static constexpr int ep = sc + kStages * kScaleBytes;
-  static constexpr int bars = ep + kMT * kEpPitch * 4;
-  static constexpr int flags = bars + 2 * kStages * 8;
-  static constexpr int table = flags + 16;        // int table[E + 1], then int offs[E + 1]
-  static constexpr int bytes_without_table = table;
 };
 
 struct Unit {
@@ -90,6 +97,7 @@ struct Unit {
 };
 
 // Unit u -> (expert, token block, tile, split); `table` and `offs` live in shared memory.
+template <int MT>
 __device__ __forceinline__ void decode_unit(const StreamArgs& A, const int* table, const int* offs,
                                             int64_t u, Unit& U) {
   int lo = 0, hi = A.E - 1;                       // largest e with table[e] <= u
@@ -98,15 +106,16 @@ __device__ __forceinline__ void decode_unit(const StreamArgs& A, const int* tabl
     if (table[mid] <= u) lo = mid; else hi = mid - 1;
   }
   U.e = lo;
-  const int64_t off0 = offs[U.e], off1 = offs[U.e + 1];
-  const int ntb = max(1, static_cast<int>((off1 - off0 + kMT - 1) / kMT));
-  const int64_t local = u - table[U.e];
-  U.tb = static_cast<int>(local % ntb);
-  const int64_t rest = local / ntb;
-  U.sp = static_cast<int>(rest % A.splits);
-  U.nt = static_cast<int>(rest / A.splits);
-  U.r0 = off0 + static_cast<int64_t>(U.tb) * kMT;
-  U.mt = static_cast<int>(off1 - U.r0 < kMT ? off1 - U.r0 : kMT);
+  const int off0 = offs[U.e], off1 = offs[U.e + 1];
+  const int ntb = max(1, (off1 - off0 + MT - 1) / MT);
+  const int local = static_cast<int>(u) - table[U.e];      // 32-bit: unit counts fit in int
+  int rest;
+  if (ntb == 1) { U.tb = 0; rest = local; }
+  else { rest = local / ntb; U.tb = local - rest * ntb; }
+  if (A.splits == 1) { U.sp = 0; U.nt = rest; }
+  else { U.nt = rest / A.splits; U.sp = rest - U.nt * A.splits; }
+  U.r0 = off0 + U.tb * MT;
+  U.mt = min(MT, off1 - static_cast<int>(U.r0));
   U.g0 = U.sp * A.stages_per_split * kGS;
   U.g1 = min(A.kg, U.g0 + A.stages_per_split * kGS);
 }
@@ -138,93 +147,33 @@ __device__ __forceinline__ int64_t gather_row(const StreamArgs& A, int64_t r) {
   return src;
 }
 
-// The copy side of the ring: a cursor over (unit, stage) that runs kStages - 1 stages ahead.
-struct Producer {
-  int64_t u;
-  Unit U;
-  int g;
-  int64_t src_row;
-  bool done;
-};
-
-__device__ __forceinline__ void producer_load_unit(const StreamArgs& A, const int* table, const int* offs,
-                                                   int64_t total, Producer& P, int lane) {
-  P.done = P.u >= total;
-  if (P.done) return;
-  decode_unit(A, table, offs, P.u, P.U);
-  P.g = P.U.g0;
-  P.src_row = lane < P.U.mt ? gather_row(A, P.U.r0 + lane) : 0;
+// Barrier over the compute warps only (the producer warp never joins it).
+__device__ __forceinline__ void compute_sync() {
+  asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
 }
 
-// Issues the stage under the cursor into its ring slot (warp-wide call) and advances the
-// cursor.  Returns false if the bounded wait for the slot gave up.
-__device__ __forceinline__ bool producer_issue(const StreamArgs& A, const CUtensorMap* tm_codes,
-                                               const CUtensorMap* tm_scales, uint8_t* smem,
-                                               uint64_t* full, uint64_t* empty, const int* table,
-                                               const int* offs, int64_t total, Producer& P,
-                                               uint32_t stage_index, int lane) {
-  if (P.done) return true;
-  const int slot = stage_index % kStages;
-  const uint32_t round = stage_index / kStages;
-  if (round > 0) {
-    bool ok = true;
-    if (lane == 0) ok = mbar_wait(&empty[slot], (round - 1) & 1);
-    if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
-  }
-  const Unit& U = P.U;
-  const int g = P.g;
-  const int gc = min(kGS, U.g1 - g);
-  uint8_t* cdst = smem + SmemLayout::codes + slot * kCodeBytes;
-  uint8_t* xdst = smem + SmemLayout::x + slot * kXBytes;
-  uint8_t* sdst = smem + SmemLayout::sc + slot * kScaleBytes;
-  const uint32_t xbytes = static_cast<uint32_t>(gc) * 64u;
-  if (lane == 0) {
-    const int64_t row_a = tile_row(A, U, 0);
-    const int64_t row_b = tile_row(A, U, kHalf);
-    uint32_t sbytes = 0;
-    if (A.scale_mode == kScaleTma) sbytes = 2 * kHalf * kGS * 2;
-    else if (A.scale_mode == kScaleBlock) sbytes = 2 * kHalf * A.kg * 2;
-    mbar_arrive_expect_tx(&full[slot], kCodeBytes + sbytes + xbytes * U.mt);
-    tma_load_2d(cdst, tm_codes, g * 4, static_cast<int32_t>(row_a), &full[slot]);
-    tma_load_2d(cdst + kHalf * 128, tm_codes, g * 4, static_cast<int32_t>(row_b), &full[slot]);
-    if (A.scale_mode == kScaleTma) {
-      tma_load_2d(sdst, tm_scales, g, static_cast<int32_t>(row_a), &full[slot]);
-      tma_load_2d(sdst + kHalf * kGS * 2, tm_scales, g, static_cast<int32_t>(row_b), &full[slot]);
-    } else if (A.scale_mode == kScaleBlock) {
-      const uint32_t blk = kHalf * A.kg * 2;
-      bulk_g2s(sdst, A.scales + row_a * A.kg, blk, &full[slot]);
-      bulk_g2s(sdst + blk, A.scales + row_b * A.kg, blk, &full[slot]);
-    }
-  }
-  __syncwarp();
-  if (lane < U.mt)
-    bulk_g2s(xdst + lane * kXPitch, A.a + P.src_row * A.K + static_cast<int64_t>(g) * 32, xbytes,
-             &full[slot]);
-  P.g += kGS;
-  if (P.g >= U.g1) {
-    P.u += gridDim.x;
-    producer_load_unit(A, table, offs, total, P, lane);
-  }
-  return true;
-}
-
+template <int MT>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
                    const __grid_constant__ CUtensorMap tmap_scales, StreamArgs A) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SmemLayout::bars);
-  uint64_t* empty = full + kStages;
-  volatile int* flags = reinterpret_cast<volatile int*>(smem + SmemLayout::flags);
-  int* table = reinterpret_cast<int*>(smem + SmemLayout::table);
+  // 1024-byte aligned base (128-byte swizzle atoms), derived by pointer arithmetic so that every
+  // pointer below stays in the shared address space (plain shared loads, not generic ones)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const Layout& L = A.L;
+  const int S = L.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off);
+  uint64_t* empty = full + S;
+  volatile int* flags = reinterpret_cast<volatile int*>(smem + L.flag_off);
+  int* table = reinterpret_cast<int*>(smem + L.table_off);
   int* offs = table + (A.E + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // Activation stages start zeroed: groups past a K tail read finite (stale or zero) values
   // that meet a zero scale.
-  for (int i = threadIdx.x; i < kStages * kXBytes / 16; i += blockDim.x)
-    reinterpret_cast<uint4*>(smem + SmemLayout::x)[i] = make_uint4(0, 0, 0, 0);
+  for (int i = threadIdx.x; i < S * L.x_bytes / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(smem + L.x_off)[i] = make_uint4(0, 0, 0, 0);
 
   // unit table: table[e] = first unit of expert e, table[E] = total; offsets copied to offs[].
   // Offsets that are not non-decreasing from 0 to rows make the launch a no-op (W4_ERR_INVALID_ARG).
@@ -239,7 +188,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         const int64_t o0 = A.offsets ? A.offsets[e] : 0;
         const int64_t o1 = A.offsets ? A.offsets[e + 1] : A.rows;
         if (o1 < o0 || o0 < 0 || o1 > A.rows) bad = true;
-        const int64_t ntb = o1 > o0 ? (o1 - o0 + kMT - 1) / kMT : 0;
+        const int64_t ntb = o1 > o0 ? (o1 - o0 + MT - 1) / MT : 0;
         cnt = static_cast<int>(ntb * A.n_tiles * A.splits);
         offs[e] = static_cast<int>(o0);
         if (e == A.E - 1) offs[A.E] = static_cast<int>(o1);
@@ -258,7 +207,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     if (bad && lane == 0) set_status(A.dev_status, W4_ERR_INVALID_ARG);
   }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kWarps);
     }
@@ -268,20 +217,62 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
   __syncthreads();
   const int64_t total_units = table[A.E];
 
-  Producer P;
-  uint32_t issued = 0;
-  if (warp == 0) {
+  if (warp == kWarps) {
+    // ------------------------------- producer -------------------------------
     if (lane == 0) {
       prefetch_tmap(&tmap_codes);
       if (A.scale_mode == kScaleTma) prefetch_tmap(&tmap_scales);
     }
-    P.u = blockIdx.x;
-    producer_load_unit(A, table, offs, total_units, P, lane);
-    for (; issued < kStages - 1 && !P.done; ++issued)
-      producer_issue(A, &tmap_codes, &tmap_scales, smem, full, empty, table, offs, total_units, P,
-                     issued, lane);
+    int slot = 0;
+    uint32_t phase = 0;        // phase of the empty barrier to wait for on the next lap
+    bool first_lap = true;
+    for (int64_t u = blockIdx.x; u < total_units; u += gridDim.x) {
+      Unit U;
+      decode_unit<MT>(A, table, offs, u, U);
+      const int64_t src_row = lane < U.mt ? gather_row(A, U.r0 + lane) : 0;
+      const int64_t row_a = tile_row(A, U, 0);
+      const int64_t row_b = tile_row(A, U, kHalf);
+      for (int g = U.g0; g < U.g1; g += kGS) {
+        if (!first_lap) {
+          bool ok = true;
+          if (lane == 0) ok = mbar_wait(&empty[slot], phase);
+          if (!__shfl_sync(0xffffffffu, ok, 0) || flags[0]) {
+            if (lane == 0) { set_status(A.dev_status, W4_ERR_TIMEOUT); flags[0] = 1; }
+            return;
+          }
+        }
+        const int gc = min(kGS, U.g1 - g);
+        uint8_t* cdst = smem + slot * kCodeBytes;
+        uint8_t* xdst = smem + L.x_off + slot * L.x_bytes;
+        uint8_t* sdst = smem + L.sc_off + slot * L.sc_bytes;
+        const uint32_t xbytes = static_cast<uint32_t>(gc) * 64u;
+        if (lane == 0) {
+          uint32_t sbytes = 0;
+          if (A.scale_mode == kScaleTma) sbytes = 2 * kHalf * kGS * 2;
+          else if (A.scale_mode == kScaleBlock) sbytes = 2 * kHalf * A.kg * 2;
+          mbar_arrive_expect_tx(&full[slot], kCodeBytes + sbytes + xbytes * U.mt);
+          tma_load_2d(cdst, &tmap_codes, g * 4, static_cast<int32_t>(row_a), &full[slot]);
+          tma_load_2d(cdst + kHalf * 128, &tmap_codes, g * 4, static_cast<int32_t>(row_b), &full[slot]);
+          if (A.scale_mode == kScaleTma) {
+            tma_load_2d(sdst, &tmap_scales, g, static_cast<int32_t>(row_a), &full[slot]);
+            tma_load_2d(sdst + kHalf * kGS * 2, &tmap_scales, g, static_cast<int32_t>(row_b), &full[slot]);
+          } else if (A.scale_mode == kScaleBlock) {
+            const uint32_t blk = kHalf * A.kg * 2;
+            bulk_g2s(sdst, A.scales + row_a * A.kg, blk, &full[slot]);
+            bulk_g2s(sdst + blk, A.scales + row_b * A.kg, blk, &full[slot]);
+          }
+        }
+        __syncwarp();
+        if (lane < U.mt)
+          bulk_g2s(xdst + lane * kXPitch, A.a + src_row * A.K + static_cast<int64_t>(g) * 32, xbytes,
+                   &full[slot]);
+        if (++slot == S) { slot = 0; if (!first_lap) phase ^= 1u; first_lap = false; }
+      }
+    }
+    return;
   }
 
+  // ------------------------------- compute warps -------------------------------
   // Rows of this thread's two A-fragment rows.  GELU gate: rlo = gate row j, rhi = up row j of
   // the same j (tile rows 8w+gid and 64+8w+gid), so the gate is applied in registers.  Otherwise
   // 16 consecutive rows per warp.
@@ -291,40 +282,34 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
   const int rhi = gelu ? rlo + kHalf : rlo + 8;
   const int r7 = rlo & 7;                       // == rhi & 7
   const int dw = (rhi - rlo) * 32;              // word distance between the two rows
-  float* ep = reinterpret_cast<float*>(smem + SmemLayout::ep);
-  uint32_t it = 0;
+  constexpr int NB = MT / 8;                    // token blocks of 8 (the MMA's n)
+  float* ep = reinterpret_cast<float*>(smem + (L.ep_off >= 0 ? L.ep_off : 0));
+  int cslot = 0;          // ring slot and mbarrier phase of the current stage
+  uint32_t cphase = 0;
   bool aborted = false;   // after a timed-out wait: skip work, keep every barrier
   for (int64_t u = blockIdx.x; u < total_units; u += gridDim.x) {
     Unit U;
-    decode_unit(A, table, offs, u, U);
+    decode_unit<MT>(A, table, offs, u, U);
     const int nblk = (U.mt + 7) >> 3;
-    float acc[2][4];
+    float acc[NB][4];
 #pragma unroll
-    for (int b = 0; b < 2; ++b)
+    for (int b = 0; b < NB; ++b)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[b][i] = 0.f;
 
-    for (int g = U.g0; g < U.g1; g += kGS, ++it) {
-      // keep the ring full: warp 0 issues the stage kStages - 1 ahead of this one
-      if (warp == 0 && !aborted && !P.done) {
-        if (!producer_issue(A, &tmap_codes, &tmap_scales, smem, full, empty, table, offs,
-                            total_units, P, issued, lane)) {
-          if (lane == 0) { set_status(A.dev_status, W4_ERR_TIMEOUT); flags[0] = 1; }
-          aborted = true;
-        }
-        ++issued;
-      }
-      const int slot = it % kStages;
-      const uint32_t round = it / kStages;
+    for (int g = U.g0; g < U.g1; g += kGS) {
+      const int slot = cslot;
+      const uint32_t phase = cphase;
+      if (++cslot == S) { cslot = 0; cphase ^= 1u; }
       const int gc = min(kGS, U.g1 - g);
-      if (!aborted && (!mbar_wait(&full[slot], round & 1) || flags[0])) {
+      if (!aborted && (!mbar_wait(&full[slot], phase) || flags[0])) {
         if (lane == 0) { set_status(A.dev_status, W4_ERR_TIMEOUT); flags[0] = 1; }
         aborted = true;
       }
       if (aborted) continue;
-      const uint32_t* cw = reinterpret_cast<const uint32_t*>(smem + SmemLayout::codes + slot * kCodeBytes);
-      const uint8_t* xs = smem + SmemLayout::x + slot * kXBytes;
-      const uint8_t* ss = smem + SmemLayout::sc + slot * kScaleBytes;
+      const uint32_t* cw = reinterpret_cast<const uint32_t*>(smem + slot * kCodeBytes);
+      const uint8_t* xs = smem + L.x_off + slot * L.x_bytes;
+      const uint8_t* ss = smem + L.sc_off + slot * L.sc_bytes;
       // scales of rows rlo / rhi for the stage's 8 groups, two bf16 per word
       uint32_t slo[4], shi[4];
       if (A.scale_mode == kScaleTma) {
@@ -355,7 +340,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           shi[p] = h0 | (h1 << 16);
         }
       }
-      // Two halves of 4 groups: dequantise rows rlo / rhi into MMA A fragments, then run the
+      // Passes of kGP groups: dequantise rows rlo / rhi into MMA A fragments, then run the
       // token blocks.  Word (row r, group gi, quad position tq) sits at chunk gi ^ (r % 8) of the
       // 128-byte row (TMA 128-byte swizzle).  Each extracted bf16 pair is two consecutive k, so
       // k-step 0 takes elements 8tq+0..3 (x pairs .x, .y) and k-step 1 elements 8tq+4..7 (.z, .w).
@@ -363,23 +348,25 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       const uint32_t* cwl = cw + rlo * 32 + tq;
       const bool mask_tail = (A.scale_mode != kScaleTma) && gc < kGS;   // TMA zero-fills past K
 #pragma unroll
-      for (int h = 0; h < kGS; h += 4) {
-        uint32_t fa[4][8];
-        float fsl[4], fsh[4];
+      for (int h = 0; h < kGS; h += kGP) {
+        uint32_t fa[kGP][8];
+        float fsl[kGP], fsh[kGP];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kGP; ++i) {
           const int gi = h + i;
           const uint32_t* pw = cwl + ((gi ^ r7) << 2);
           const uint32_t wlo = pw[0];
           const uint32_t whi = pw[dw];
-          fa[i][0] = nibbles_to_bf16x2(wlo);        // k-step 0: elements (0,1) | (2,3)
-          fa[i][1] = nibbles_to_bf16x2(whi);
-          fa[i][2] = nibbles_to_bf16x2(wlo >> 4);
-          fa[i][3] = nibbles_to_bf16x2(whi >> 4);
-          fa[i][4] = nibbles_to_bf16x2(wlo >> 8);   // k-step 1: elements (4,5) | (6,7)
-          fa[i][5] = nibbles_to_bf16x2(whi >> 8);
-          fa[i][6] = nibbles_to_bf16x2(wlo >> 12);
-          fa[i][7] = nibbles_to_bf16x2(whi >> 12);
+          // biased codes 128 + u (exact in bf16); the -136 * sum(x) term comes from one MMA per
+          // k-step with the constant A = -136, so q * x = (128 + u) * x - 136 * x overall
+          fa[i][0] = nibbles_to_bf16x2_biased(wlo);        // k-step 0: elements (0,1) | (2,3)
+          fa[i][1] = nibbles_to_bf16x2_biased(whi);
+          fa[i][2] = nibbles_to_bf16x2_biased(wlo >> 4);
+          fa[i][3] = nibbles_to_bf16x2_biased(whi >> 4);
+          fa[i][4] = nibbles_to_bf16x2_biased(wlo >> 8);   // k-step 1: elements (4,5) | (6,7)
+          fa[i][5] = nibbles_to_bf16x2_biased(whi >> 8);
+          fa[i][6] = nibbles_to_bf16x2_biased(wlo >> 12);
+          fa[i][7] = nibbles_to_bf16x2_biased(whi >> 12);
           const uint32_t sl = (gi & 1) ? (slo[gi >> 1] & 0xFFFF0000u) : (slo[gi >> 1] << 16);
           const uint32_t sh = (gi & 1) ? (shi[gi >> 1] & 0xFFFF0000u) : (shi[gi >> 1] << 16);
           fsl[i] = __uint_as_float(sl);
@@ -387,17 +374,20 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           if (mask_tail && gi >= gc) { fsl[i] = 0.f; fsh[i] = 0.f; }   // past the K range
         }
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NB; ++b) {
           if (b < nblk) {
             const uint8_t* xrow = xs + (b * 8 + gid) * kXPitch + tq * 16;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < kGP; ++i) {
               const uint4 xv = *reinterpret_cast<const uint4*>(xrow + (h + i) * 64);
               const uint32_t a0[4] = {fa[i][0], fa[i][1], fa[i][2], fa[i][3]};
               const uint32_t a1[4] = {fa[i][4], fa[i][5], fa[i][6], fa[i][7]};
+              const uint32_t ac[4] = {kMinus136x2, kMinus136x2, kMinus136x2, kMinus136x2};
               float d[4];
               const float z[4] = {0.f, 0.f, 0.f, 0.f};
-              mma_bf16_16816(d, a0, xv.x, xv.y, z);
+              mma_bf16_16816(d, ac, xv.x, xv.y, z);
+              mma_bf16_16816(d, ac, xv.z, xv.w, d);
+              mma_bf16_16816(d, a0, xv.x, xv.y, d);
               mma_bf16_16816(d, a1, xv.z, xv.w, d);
               acc[b][0] = fmaf(fsl[i], d[0], acc[b][0]);
               acc[b][1] = fmaf(fsl[i], d[1], acc[b][1]);
@@ -416,7 +406,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       // straight from registers: thread holds rows rlo / rhi for tokens 2tq, 2tq + 1 of each block
       if (!aborted) {
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NB; ++b) {
           if (b < nblk) {
             const int t0 = b * 8 + 2 * tq;
             if (gelu) {
@@ -447,7 +437,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     // split-K (dense, no gate): float32 partials through shared memory, then the last CTA of the
     // tile reduces them in split order
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NB; ++b) {
       if (b < nblk) {
         const int t0 = b * 8 + 2 * tq;
         ep[t0 * kEpPitch + rlo] = acc[b][0];
@@ -456,18 +446,18 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         ep[(t0 + 1) * kEpPitch + rhi] = acc[b][3];
       }
     }
-    __syncthreads();
+    compute_sync();
     const int ctid = threadIdx.x;
     const int n0 = U.nt * kBN;
     if (!flags[0]) {
-      for (int idx = ctid; idx < U.mt * kBN; idx += kThreads) {
+      for (int idx = ctid; idx < U.mt * kBN; idx += kWarps * 32) {
         const int t = idx / kBN, c = idx % kBN;
         if (n0 + c < A.N)
           A.partial[(static_cast<int64_t>(U.sp) * A.rows + U.r0 + t) * A.N + n0 + c] = ep[t * kEpPitch + c];
       }
     }
     __threadfence();
-    __syncthreads();
+    compute_sync();
     if (ctid == 0) {
       int last = 0;
       if (!flags[0]) {
@@ -478,10 +468,10 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       }
       flags[1] = last;
     }
-    __syncthreads();
+    compute_sync();
     if (flags[1]) {
       __threadfence();
-      for (int idx = ctid; idx < U.mt * kBN; idx += kThreads) {
+      for (int idx = ctid; idx < U.mt * kBN; idx += kWarps * 32) {
         const int t = idx / kBN, c = idx % kBN;
         if (n0 + c < A.N) {
           float sum = 0.f;
@@ -491,7 +481,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         }
       }
     }
-    __syncthreads();
+    compute_sync();
   }
 }
 
@@ -541,25 +531,53 @@ static bool encode_scales_map(CUtensorMap* m, const uint16_t* scales, int64_t ro
   return r == CUDA_SUCCESS;
 }
 
-static size_t stream_smem_bytes(int E) {
-  return w4::SmemLayout::bytes_without_table + static_cast<size_t>(E + 1) * 8 + 1024;
+// Ring depth and offsets for one launch: as many stages (up to kMaxStages) as fit the per-CTA
+// shared-memory budget next to the fixed parts.
+static w4::Layout make_layout(int MT, int scale_mode, int kg, int E, bool split) {
+  w4::Layout L{};
+  L.x_bytes = MT * w4::kXPitch;
+  L.sc_bytes = scale_mode == w4::kScaleTma ? 2 * w4::kHalf * w4::kGS * 2
+             : scale_mode == w4::kScaleBlock ? 2 * w4::kHalf * kg * 2 : 16;
+  L.sc_bytes = (L.sc_bytes + 127) & ~127;
+  const int ep_bytes = split ? MT * w4::kEpPitch * 4 : 0;
+  const int fixed = ep_bytes + 2 * w4::kMaxStages * 8 + 16 + (E + 1) * 8 + 1024;   // + alignment slack
+  const int per_stage = w4::kCodeBytes + L.x_bytes + L.sc_bytes;
+  int S = (w4::kSmemPerCta - fixed) / per_stage;
+  if (S > w4::kMaxStages) S = w4::kMaxStages;
+  L.stages = S;
+  L.x_off = S * w4::kCodeBytes;
+  L.sc_off = L.x_off + S * L.x_bytes;
+  int off = L.sc_off + S * L.sc_bytes;
+  L.ep_off = split ? off : -1;
+  off += ep_bytes;
+  L.bar_off = (off + 7) & ~7;
+  off = L.bar_off + 2 * S * 8;
+  L.flag_off = off;
+  off += 16;
+  L.table_off = off;
+  off += (E + 1) * 8;
+  L.total = off + 1024;
+  return L;
 }
 
 struct StreamPlan {
-  int splits, stages_per_split, n_tiles;
+  int splits, stages_per_split, n_tiles, MT;
 };
 
 static StreamPlan plan_stream(int64_t rows, int N, int K, int E, int epi, bool dense, int sm_count) {
   StreamPlan p;
   const int kg = K / 32;
   const int kstages = (kg + w4::kGS - 1) / w4::kGS;
+  // token block: 8 rows when experts hold few rows on average (keeps the activation ring small and
+  // the weight ring deep), else 16
+  p.MT = (rows <= 6LL * E) ? 8 : 16;
   p.n_tiles = (epi == W4_EPI_GELU_GATE) ? ((N / 2) + w4::kHalf - 1) / w4::kHalf
                                         : (N + w4::kBN - 1) / w4::kBN;
   p.splits = 1;
   if (dense) {
     // split K while the units do not fill the CTAs four times over and the float32 partials
     // stay below ~1/8 of the weight bytes
-    const int64_t ntb = (rows + w4::kMT - 1) / w4::kMT;
+    const int64_t ntb = (rows + p.MT - 1) / p.MT;
     const double wbytes = static_cast<double>(N) * K * 0.5625;
     while (p.splits * 2 <= kstages && ntb * p.n_tiles * p.splits < 4LL * w4::kCtasPerSm * sm_count &&
            static_cast<double>(p.splits * 2) * rows * N * 8.0 <= wbytes / 8.0)
@@ -573,10 +591,29 @@ static StreamPlan plan_stream(int64_t rows, int N, int K, int E, int epi, bool d
 size_t w4_stream_workspace_bytes(int64_t rows, int N, int K, int E, int epi, bool dense, int sm_count) {
   StreamPlan p = plan_stream(rows, N, K, E, epi, dense, sm_count);
   if (p.splits == 1) return 0;
-  const int64_t ntb = (rows + w4::kMT - 1) / w4::kMT;
+  const int64_t ntb = (rows + p.MT - 1) / p.MT;
   size_t b = static_cast<size_t>(p.splits) * rows * N * sizeof(float);
   b = (b + 255) & ~size_t(255);
   return b + static_cast<size_t>(ntb * p.n_tiles) * sizeof(int32_t);
+}
+
+template <int MT>
+static w4_status launch_mt(const CUtensorMap& tmap, const CUtensorMap& smap, const w4::StreamArgs& A,
+                           int sm_count, cudaStream_t stream) {
+  static int attr_done[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(w4::stream_gemm_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             w4::kSmemPerCta) != cudaSuccess)
+      return W4_ERR_CUDA;
+    if (cudaFuncSetAttribute(w4::stream_gemm_kernel<MT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+      return W4_ERR_CUDA;
+    attr_done[dev] = 1;
+  }
+  w4::stream_gemm_kernel<MT><<<sm_count * w4::kCtasPerSm, w4::kThreads, A.L.total, stream>>>(tmap, smap, A);
+  return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
 w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int k_div,
@@ -606,6 +643,8 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
   } else {
     A.scale_mode = w4::kScaleLdg;
   }
+  A.L = make_layout(p.MT, A.scale_mode, A.kg, E, p.splits > 1);
+  if (A.L.stages < 2) return W4_ERR_UNSUPPORTED;
   if (p.splits > 1) {
     const size_t need = w4_stream_workspace_bytes(rows, N, K, E, epi, dense, sm_count);
     if (ws == nullptr || ws_bytes < need) return W4_ERR_WORKSPACE;
@@ -621,19 +660,6 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
   if (A.scale_mode == w4::kScaleTma &&
       !encode_scales_map(&smap, scales, static_cast<int64_t>(E) * N, A.kg))
     return W4_ERR_CUDA;
-  const size_t smem = stream_smem_bytes(E);
-  static int attr_done[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(w4::stream_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(stream_smem_bytes(1024))) != cudaSuccess)
-      return W4_ERR_CUDA;
-    if (cudaFuncSetAttribute(w4::stream_gemm_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
-      return W4_ERR_CUDA;
-    attr_done[dev] = 1;
-  }
-  w4::stream_gemm_kernel<<<sm_count * w4::kCtasPerSm, w4::kThreads, smem, stream>>>(tmap, smap, A);
-  return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+  return p.MT == 8 ? launch_mt<8>(tmap, smap, A, sm_count, stream)
+                   : launch_mt<16>(tmap, smap, A, sm_count, stream);
 }
