@@ -96,9 +96,9 @@ w4_status w4_repack(const uint16_t* w, int64_t rows, int64_t K, uint32_t* codes,
  *   M >= 0, N >= 1, K >= 32 with K % 32 == 0.
  *   workspace, workspace_bytes: device scratch of at least
  *            w4_workspace_bytes(W4_OP_LINEAR, M, N, K, 1, 1) bytes (may be NULL when that is 0).
- *            Its counter words must be zero before the first use (e.g. a fresh cudaMemset);
- *            every call that completes leaves them zero again.  Calls sharing one workspace must
- *            not overlap on the GPU.
+ *            Its contents need no preparation (the call clears the part it relies on, with a
+ *            cudaMemsetAsync on `stream`).  Calls sharing one workspace must not overlap on the
+ *            GPU.
  * y[m, n] = bf16(sum_k x[m, k] * s[n, k/32] * q[n, k]) with float32 accumulation.
  */
 w4_status w4a16_linear(const uint16_t* x, const uint32_t* codes, const uint16_t* scales,

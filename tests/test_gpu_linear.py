@@ -77,3 +77,19 @@ def test_repeat_calls_are_deterministic():
     y1 = host_bf16_bits(_run(case))
     y2 = host_bf16_bits(_run(case))
     assert np.array_equal(y1, y2)
+
+
+def test_workspace_reused_across_shapes_with_stale_contents():
+    """One workspace filled with garbage and shared by split-K calls of different shapes."""
+    from w4a16_group_quantized_w4_b200 import _lib
+    shapes = [(1, 14336, 4096), (4, 14336, 4096), (16, 14336, 4096), (3, 2048, 2816), (1, 14336, 4096)]
+    need = max(api.w4_workspace_bytes(_lib.W4_OP_LINEAR, M, N, K, 1, 1) for M, N, K in shapes)
+    assert need > 0
+    ws = torch.full((need,), 0xA5, dtype=torch.uint8, device="cuda")
+    for i, (M, N, K) in enumerate(shapes):
+        case = synth.dense_case(M, N, K, 0.01, 1e-4, seed=40 + i)
+        y = api.w4a16_linear(dev_bf16(case.x), dev_u32(case.codes), dev_bf16(case.scales), ws=ws)
+        torch.cuda.synchronize()
+        cols = np.arange(0, N, 97)
+        ref = linear.w4a16_linear_rows(case.x, case.codes, case.scales, cols)
+        assert_rows_close(host_f64(y)[:, cols], ref)

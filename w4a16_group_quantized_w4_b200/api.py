@@ -47,8 +47,8 @@ _WS: dict = {}
 
 
 def workspace(nbytes: int, device) -> torch.Tensor | None:
-    """A zero-initialised scratch buffer of at least nbytes, cached per device (counters in it
-    return to zero after every completed call, so it is reused as is)."""
+    """A scratch buffer of at least nbytes, cached per device and shared by calls on it (the
+    library clears what it relies on, so contents left by earlier calls do not matter)."""
     if nbytes == 0:
         return None
     key = torch.device(device)

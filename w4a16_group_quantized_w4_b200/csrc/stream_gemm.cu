@@ -588,13 +588,17 @@ static StreamPlan plan_stream(int64_t rows, int N, int K, int E, int epi, bool d
   return p;
 }
 
+// Split-K workspace: the per-tile arrival counters first (cleared by every launch), then the
+// float32 partials [splits, rows, N].
+static size_t counters_bytes(const StreamPlan& p, int64_t rows) {
+  const int64_t ntb = (rows + p.MT - 1) / p.MT;
+  return (static_cast<size_t>(ntb * p.n_tiles) * sizeof(int32_t) + 255) & ~size_t(255);
+}
+
 size_t w4_stream_workspace_bytes(int64_t rows, int N, int K, int E, int epi, bool dense, int sm_count) {
   StreamPlan p = plan_stream(rows, N, K, E, epi, dense, sm_count);
   if (p.splits == 1) return 0;
-  const int64_t ntb = (rows + p.MT - 1) / p.MT;
-  size_t b = static_cast<size_t>(p.splits) * rows * N * sizeof(float);
-  b = (b + 255) & ~size_t(255);
-  return b + static_cast<size_t>(ntb * p.n_tiles) * sizeof(int32_t);
+  return counters_bytes(p, rows) + static_cast<size_t>(p.splits) * rows * N * sizeof(float);
 }
 
 template <int MT>
@@ -648,10 +652,11 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
   if (p.splits > 1) {
     const size_t need = w4_stream_workspace_bytes(rows, N, K, E, epi, dense, sm_count);
     if (ws == nullptr || ws_bytes < need) return W4_ERR_WORKSPACE;
-    size_t pb = static_cast<size_t>(p.splits) * rows * N * sizeof(float);
-    pb = (pb + 255) & ~size_t(255);
-    A.partial = static_cast<float*>(ws);
-    A.counters = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + pb);
+    const size_t cb = counters_bytes(p, rows);
+    A.counters = static_cast<int32_t*>(ws);
+    A.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + cb);
+    // the arrival counters must start at zero whatever the workspace held before
+    if (rows > 0 && cudaMemsetAsync(ws, 0, cb, stream) != cudaSuccess) return W4_ERR_CUDA;
   }
   if (rows == 0) return W4_OK;
   CUtensorMap tmap, smap;
