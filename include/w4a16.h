@@ -161,6 +161,28 @@ w4_status moe_w4a16_gmm(const uint16_t* a, const int32_t* a_row_of_pair, int32_t
 w4_status moe_combine(const uint16_t* o, const float* topk_w, const int32_t* pair_pos,
                       int32_t T, int32_t k, int32_t H, uint16_t* y, void* stream);
 
+/*
+ * w4a16_linear_noalloc -- w4a16_linear for callers that cannot allocate device memory.
+ * (No counterpart on the pages: an interface addition of this library.)
+ *
+ * Same arguments, result and accuracy as w4a16_linear, without a workspace: when K is split
+ * across CTAs the float32 partials and arrival counters live in a file-scope device array of
+ * 8 MiB (8388608 bytes) that every GPU loading the library keeps until process exit.  Callers
+ * that are handed only their input and output buffers (a plugin inside a framework that owns all
+ * device memory through its own pool, or a runtime held to a fixed memory budget) can call it
+ * without cudaMalloc, which would bypass the pool and synchronise the device.
+ *   - Returns W4_ERR_WORKSPACE when the sizes need more scratch than 8 MiB
+ *     (w4_workspace_bytes(W4_OP_LINEAR, M, N, K, 1, 1) > 8388608).
+ *   - The first call on a device looks up the array's device address (once per device); make
+ *     that first call before any stream capture.
+ *   - Every call reuses the same array (clearing its arrival counters with a cudaMemsetAsync on
+ *     `stream`): calls that overlap on the GPU race and must be ordered by the caller (one
+ *     stream, or events).
+ *   - Allocates nothing: no cudaMalloc/cudaFree, no allocating library routine.
+ */
+w4_status w4a16_linear_noalloc(const uint16_t* x, const uint32_t* codes, const uint16_t* scales,
+                               uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream);
+
 /* Workspace bytes an entry point needs for the given sizes (0 when it needs none). */
 size_t w4_workspace_bytes(int32_t op, int64_t M_or_T, int64_t N, int64_t K, int32_t E, int32_t k);
 

@@ -103,6 +103,27 @@ def w4a16_linear(x, codes, scales, y=None, ws=None, stream=None):
     return y
 
 
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def w4a16_linear_noalloc(x, codes, scales, y=None, stream=None):
+    """Like w4a16_linear, but never needs a workspace: split-K scratch comes from the library's
+    fixed 8 MiB device array (for callers that cannot allocate device memory).  Calls that
+    overlap on the GPU share that array and must be ordered by the caller."""
+    lib = _lib.load()
+    M, K = x.shape
+    N = codes.shape[0]
+    dev = x.device
+    _need("x", x, torch.bfloat16)
+    _need("codes", codes, torch.int32, (N, K // 8), dev)
+    _need("scales", scales, torch.bfloat16, (N, K // 32), dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev) if y is None else y
+    _need("y", y, torch.bfloat16, (M, N), dev)
+    _lib.check("w4a16_linear_noalloc", lib.w4a16_linear_noalloc(_p(x), _p(codes), _p(scales), _p(y),
+                                                                M, N, K, _s(stream)))
+    return y
+
+
 class Routing:
     __slots__ = ("topk_ids", "topk_w", "expert_offsets", "sorted_pair", "pair_pos")
 
