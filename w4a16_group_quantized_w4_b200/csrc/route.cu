@@ -20,9 +20,10 @@
 
 namespace w4 {
 
-constexpr int kRouteWarps = 8;                 // warps per CTA
+constexpr int kRouteWarps = 8;                 // warps per CTA in the two-launch path
+constexpr int kFusedWarps = 32;                // warps of the single-CTA path
 constexpr int kRouteTokensPerCta = 64;         // tokens per CTA in the two-launch path
-constexpr int kMaxEPerLane = 32;               // E <= 1024
+constexpr int kFusedMaxT = 128;                // largest T routed by the single-CTA path
 
 struct RouteArgs {
   const float* logits;
@@ -34,6 +35,7 @@ struct RouteArgs {
   int32_t* pair_pos;
   int32_t* hist;       // [num_ctas][E] per-CTA counts (workspace)
   int tokens_per_cta;
+  int scatter_warps;    // warps taking part in the scatter (shared scratch scales with it)
 };
 
 __device__ __forceinline__ bool better(float v, int i, float w, int j) {
@@ -41,28 +43,28 @@ __device__ __forceinline__ bool better(float v, int i, float w, int j) {
 }
 
 // Top-k for tokens [t0, t1) of this CTA; accumulates counts into s_cnt[E] (shared).
+// PL = logits per lane (E <= 32 * PL); lane l holds experts c * 32 + l.
+template <int PL>
 __device__ void topk_tokens(const RouteArgs& A, int t0, int t1, int* s_cnt) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int per_lane = (A.E + 31) >> 5;
   for (int t = t0 + warp; t < t1; t += nwarps) {
-    float v[kMaxEPerLane];
+    float v[PL];
     const float* row = A.logits + static_cast<int64_t>(t) * A.E;
 #pragma unroll
-    for (int c = 0; c < kMaxEPerLane; ++c) {
+    for (int c = 0; c < PL; ++c) {
       const int e = c * 32 + lane;
-      v[c] = (c < per_lane && e < A.E) ? row[e] : -INFINITY;
+      v[c] = e < A.E ? __ldg(row + e) : -INFINITY;
     }
     uint32_t taken = 0;
-    float sel_v = 0.f;
+    float sel_v = 0.f, top = 0.f;
     int sel_e = 0;
-    float top = 0.f;
     for (int j = 0; j < A.k; ++j) {
       float bv = -INFINITY;
       int be = 0x7FFFFFFF;
 #pragma unroll
-      for (int c = 0; c < kMaxEPerLane; ++c) {
+      for (int c = 0; c < PL; ++c) {
         const int e = c * 32 + lane;
-        if (c < per_lane && e < A.E && !((taken >> c) & 1u) && better(v[c], e, bv, be)) {
+        if (e < A.E && !((taken >> c) & 1u) && better(v[c], e, bv, be)) {
           bv = v[c];
           be = e;
         }
@@ -91,15 +93,18 @@ __device__ void topk_tokens(const RouteArgs& A, int t0, int t1, int* s_cnt) {
 
 // Positions for pairs [p0, p1) given this CTA's per-expert base s_base[E] (shared).
 // s_wcnt: [nwarps][E] shared scratch.
+// nwarps warps take part (the others only join the CTA barriers).
 __device__ void scatter_pairs(const RouteArgs& A, int64_t p0, int64_t p1, const int* s_base,
-                              int* s_wcnt) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+                              int* s_wcnt, int nwarps) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const bool active = warp < nwarps;
   const int64_t n = p1 - p0;
   const int64_t per_warp = (n + nwarps - 1) / nwarps;
-  const int64_t w0 = p0 + warp * per_warp;
-  const int64_t w1 = min(p1, w0 + per_warp);
-  int* mycnt = s_wcnt + warp * A.E;
-  for (int e = lane; e < A.E; e += 32) mycnt[e] = 0;
+  const int64_t w0 = p0 + (active ? warp : nwarps) * per_warp;
+  const int64_t w1 = active ? min(p1, w0 + per_warp) : w0;
+  int* mycnt = s_wcnt + (active ? warp : 0) * A.E;
+  if (active)
+    for (int e = lane; e < A.E; e += 32) mycnt[e] = 0;
   __syncwarp();
   for (int64_t p = w0 + lane; p - lane < w1; p += 32) {
     int e = p < w1 ? A.topk_ids[p] : -1;
@@ -141,15 +146,24 @@ __device__ void scatter_pairs(const RouteArgs& A, int64_t p0, int64_t p1, const 
   }
 }
 
+__device__ __forceinline__ void topk_dispatch(const RouteArgs& A, int t0, int t1, int* s_cnt) {
+  if (A.E <= 32) topk_tokens<1>(A, t0, t1, s_cnt);
+  else if (A.E <= 64) topk_tokens<2>(A, t0, t1, s_cnt);
+  else if (A.E <= 128) topk_tokens<4>(A, t0, t1, s_cnt);
+  else if (A.E <= 256) topk_tokens<8>(A, t0, t1, s_cnt);
+  else if (A.E <= 512) topk_tokens<16>(A, t0, t1, s_cnt);
+  else topk_tokens<32>(A, t0, t1, s_cnt);
+}
+
 // One CTA does everything (small T).
-__global__ void __launch_bounds__(kRouteWarps * 32) route_fused_kernel(RouteArgs A) {
+__global__ void __launch_bounds__(kFusedWarps * 32) route_fused_kernel(RouteArgs A) {
   extern __shared__ int smem[];
   int* s_cnt = smem;                     // [E]
   int* s_base = s_cnt + A.E;             // [E]
   int* s_wcnt = s_base + A.E;            // [nwarps][E]
   for (int e = threadIdx.x; e < A.E; e += blockDim.x) s_cnt[e] = 0;
   __syncthreads();
-  topk_tokens(A, 0, A.T, s_cnt);
+  topk_dispatch(A, 0, A.T, s_cnt);
   __syncthreads();
   if (threadIdx.x == 0) {
     int run = 0;
@@ -161,8 +175,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_fused_kernel(RouteArgs
     A.expert_offsets[A.E] = run;
   }
   __syncthreads();
-  __threadfence_block();
-  scatter_pairs(A, 0, static_cast<int64_t>(A.T) * A.k, s_base, s_wcnt);
+  scatter_pairs(A, 0, static_cast<int64_t>(A.T) * A.k, s_base, s_wcnt, A.scatter_warps);
 }
 
 __global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(RouteArgs A) {
@@ -172,7 +185,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(RouteArgs 
   __syncthreads();
   const int t0 = blockIdx.x * A.tokens_per_cta;
   const int t1 = min(A.T, t0 + A.tokens_per_cta);
-  topk_tokens(A, t0, t1, s_cnt);
+  topk_dispatch(A, t0, t1, s_cnt);
   __syncthreads();
   for (int e = threadIdx.x; e < A.E; e += blockDim.x) A.hist[blockIdx.x * A.E + e] = s_cnt[e];
 }
@@ -211,13 +224,15 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_scatter_kernel(RouteAr
   __syncthreads();
   const int64_t p0 = static_cast<int64_t>(blockIdx.x) * A.tokens_per_cta * A.k;
   const int64_t p1 = min(static_cast<int64_t>(A.T) * A.k, p0 + static_cast<int64_t>(A.tokens_per_cta) * A.k);
-  scatter_pairs(A, p0, p1, s_base, s_wcnt);
+  scatter_pairs(A, p0, p1, s_base, s_wcnt, A.scatter_warps);
 }
 
 // ------------------------------------------------------------------------------------------
 // combine: y[t] = sum_j w[t, j] * o[pair_pos[t*k + j]], float32 in slot order, bf16 out.
-// One thread per 8 consecutive features (16-byte loads and stores).
+// One thread per 8 consecutive features (16-byte loads and stores); the k row indices and
+// weights are fetched first so that the k row loads are in flight together.
 // ------------------------------------------------------------------------------------------
+template <int KMAX>
 __global__ void __launch_bounds__(128) combine_kernel(const uint16_t* __restrict__ o,
                                                       const float* __restrict__ topk_w,
                                                       const int32_t* __restrict__ pair_pos,
@@ -225,19 +240,37 @@ __global__ void __launch_bounds__(128) combine_kernel(const uint16_t* __restrict
   const int t = blockIdx.x;
   const int h8 = blockIdx.y * blockDim.x + threadIdx.x;
   if (t >= T || h8 * 8 >= H) return;
+  const int64_t T_k = static_cast<int64_t>(T) * k;
+  int64_t row[KMAX];
+  float wj[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    row[j] = -1;
+    wj[j] = 0.f;
+    if (j < k) {
+      row[j] = __ldg(pair_pos + static_cast<int64_t>(t) * k + j);
+      wj[j] = __ldg(topk_w + static_cast<int64_t>(t) * k + j);
+    }
+  }
+  uint4 v[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    v[j] = make_uint4(0, 0, 0, 0);
+    if (j < k && row[j] >= 0 && row[j] < T_k)           // not a valid permutation entry: skip
+      v[j] = ldg_stream128(o + row[j] * H + h8 * 8);
+  }
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  for (int j = 0; j < k; ++j) {
-    const float wj = topk_w[static_cast<int64_t>(t) * k + j];
-    const int64_t row = pair_pos[static_cast<int64_t>(t) * k + j];
-    if (row < 0 || row >= static_cast<int64_t>(T) * k) continue;   // not a valid permutation entry
-    const uint4 v = ldg_stream128(o + row * H + h8 * 8);
-    const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      acc[2 * i] = fmaf(wj, bf16_lo_to_f32(vv[i]), acc[2 * i]);
-      acc[2 * i + 1] = fmaf(wj, bf16_hi_to_f32(vv[i]), acc[2 * i + 1]);
+  for (int j = 0; j < KMAX; ++j) {
+    if (j < k) {
+      const uint32_t vv[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = fmaf(wj[j], bf16_lo_to_f32(vv[i]), acc[2 * i]);
+        acc[2 * i + 1] = fmaf(wj[j], bf16_hi_to_f32(vv[i]), acc[2 * i + 1]);
+      }
     }
   }
   uint4 out;
@@ -257,17 +290,23 @@ __global__ void __launch_bounds__(128) combine_kernel(const uint16_t* __restrict
 static int route_num_ctas(int T) { return (T + w4::kRouteTokensPerCta - 1) / w4::kRouteTokensPerCta; }
 
 size_t w4_route_workspace_bytes(int T, int E) {
-  if (T <= w4::kRouteTokensPerCta * 4) return 0;   // fused single-CTA path
+  if (T <= w4::kFusedMaxT) return 0;   // fused single-CTA path
   return static_cast<size_t>(route_num_ctas(T)) * E * sizeof(int32_t);
+}
+
+// Warps taking part in the scatter: (2 + warps) * E ints must stay within 48 KB of shared memory.
+static int scatter_warps_for(int E, int max_warps) {
+  int w = 12288 / E - 2;
+  if (w > max_warps) w = max_warps;
+  return w < 1 ? 1 : w;
 }
 
 w4_status w4_launch_route(const float* logits, int T, int E, int k, int32_t* ids, float* w,
                           int32_t* offsets, int32_t* sorted_pair, int32_t* pair_pos, void* ws,
                           size_t ws_bytes, cudaStream_t stream) {
   w4::RouteArgs A{logits, T, E, k, ids, w, offsets, sorted_pair, pair_pos, nullptr,
-                  w4::kRouteTokensPerCta};
+                  w4::kRouteTokensPerCta, 1};
   const int threads = w4::kRouteWarps * 32;
-  const size_t smem = static_cast<size_t>(2 + w4::kRouteWarps) * E * sizeof(int);
   // (2 + warps) * E ints <= 40 KB for E <= 1024: within the default shared-memory limit
   if (T == 0) {
     // offsets are all zero
@@ -275,10 +314,14 @@ w4_status w4_launch_route(const float* logits, int T, int E, int k, int32_t* ids
     return W4_OK;
   }
   if (w4_route_workspace_bytes(T, E) == 0) {
-    w4::route_fused_kernel<<<1, threads, smem, stream>>>(A);
+    A.scatter_warps = scatter_warps_for(E, w4::kFusedWarps);
+    const size_t smem = static_cast<size_t>(2 + A.scatter_warps) * E * sizeof(int);
+    w4::route_fused_kernel<<<1, w4::kFusedWarps * 32, smem, stream>>>(A);
   } else {
     if (ws == nullptr || ws_bytes < w4_route_workspace_bytes(T, E)) return W4_ERR_WORKSPACE;
     A.hist = static_cast<int32_t*>(ws);
+    A.scatter_warps = scatter_warps_for(E, w4::kRouteWarps);
+    const size_t smem = static_cast<size_t>(2 + A.scatter_warps) * E * sizeof(int);
     const int nctas = route_num_ctas(T);
     w4::route_topk_kernel<<<nctas, threads, E * sizeof(int), stream>>>(A);
     if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
@@ -292,6 +335,7 @@ w4_status w4_launch_combine(const uint16_t* o, const float* topk_w, const int32_
   if (T == 0) return W4_OK;
   const int threads = 128;
   dim3 grid(T, (H / 8 + threads - 1) / threads);
-  w4::combine_kernel<<<grid, threads, 0, stream>>>(o, topk_w, pair_pos, T, k, H, y);
+  if (k <= 8) w4::combine_kernel<8><<<grid, threads, 0, stream>>>(o, topk_w, pair_pos, T, k, H, y);
+  else w4::combine_kernel<32><<<grid, threads, 0, stream>>>(o, topk_w, pair_pos, T, k, H, y);
   return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }

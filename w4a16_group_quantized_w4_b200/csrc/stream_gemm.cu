@@ -38,7 +38,10 @@
 namespace w4 {
 
 #ifndef W4_STREAM_GROUPS_PER_PASS
-#define W4_STREAM_GROUPS_PER_PASS 2           // groups dequantised into registers at a time
+#define W4_STREAM_GROUPS_PER_PASS 4           // groups dequantised into registers at a time
+#endif
+#ifndef W4_STREAM_BIASED
+#define W4_STREAM_BIASED 0                    // 1: codes as 128 + u plus a -136 MMA; 0: u - 8 by fma
 #endif
 
 constexpr int kMaxStages = 6;
@@ -359,14 +362,20 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           const uint32_t whi = pw[dw];
           // biased codes 128 + u (exact in bf16); the -136 * sum(x) term comes from one MMA per
           // k-step with the constant A = -136, so q * x = (128 + u) * x - 136 * x overall
-          fa[i][0] = nibbles_to_bf16x2_biased(wlo);        // k-step 0: elements (0,1) | (2,3)
-          fa[i][1] = nibbles_to_bf16x2_biased(whi);
-          fa[i][2] = nibbles_to_bf16x2_biased(wlo >> 4);
-          fa[i][3] = nibbles_to_bf16x2_biased(whi >> 4);
-          fa[i][4] = nibbles_to_bf16x2_biased(wlo >> 8);   // k-step 1: elements (4,5) | (6,7)
-          fa[i][5] = nibbles_to_bf16x2_biased(whi >> 8);
-          fa[i][6] = nibbles_to_bf16x2_biased(wlo >> 12);
-          fa[i][7] = nibbles_to_bf16x2_biased(whi >> 12);
+#if W4_STREAM_BIASED
+#define W4_DEQ nibbles_to_bf16x2_biased
+#else
+#define W4_DEQ nibbles_to_bf16x2
+#endif
+          fa[i][0] = W4_DEQ(wlo);        // k-step 0: elements (0,1) | (2,3)
+          fa[i][1] = W4_DEQ(whi);
+          fa[i][2] = W4_DEQ(wlo >> 4);
+          fa[i][3] = W4_DEQ(whi >> 4);
+          fa[i][4] = W4_DEQ(wlo >> 8);   // k-step 1: elements (4,5) | (6,7)
+          fa[i][5] = W4_DEQ(whi >> 8);
+          fa[i][6] = W4_DEQ(wlo >> 12);
+          fa[i][7] = W4_DEQ(whi >> 12);
+#undef W4_DEQ
           const uint32_t sl = (gi & 1) ? (slo[gi >> 1] & 0xFFFF0000u) : (slo[gi >> 1] << 16);
           const uint32_t sh = (gi & 1) ? (shi[gi >> 1] & 0xFFFF0000u) : (shi[gi >> 1] << 16);
           fsl[i] = __uint_as_float(sl);
@@ -382,12 +391,16 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
               const uint4 xv = *reinterpret_cast<const uint4*>(xrow + (h + i) * 64);
               const uint32_t a0[4] = {fa[i][0], fa[i][1], fa[i][2], fa[i][3]};
               const uint32_t a1[4] = {fa[i][4], fa[i][5], fa[i][6], fa[i][7]};
-              const uint32_t ac[4] = {kMinus136x2, kMinus136x2, kMinus136x2, kMinus136x2};
               float d[4];
               const float z[4] = {0.f, 0.f, 0.f, 0.f};
+#if W4_STREAM_BIASED
+              const uint32_t ac[4] = {kMinus136x2, kMinus136x2, kMinus136x2, kMinus136x2};
               mma_bf16_16816(d, ac, xv.x, xv.y, z);
               mma_bf16_16816(d, ac, xv.z, xv.w, d);
               mma_bf16_16816(d, a0, xv.x, xv.y, d);
+#else
+              mma_bf16_16816(d, a0, xv.x, xv.y, z);
+#endif
               mma_bf16_16816(d, a1, xv.z, xv.w, d);
               acc[b][0] = fmaf(fsl[i], d[0], acc[b][0]);
               acc[b][1] = fmaf(fsl[i], d[1], acc[b][1]);
