@@ -22,6 +22,21 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
                                 const int32_t* offsets, int E, int64_t rows, int N, int K, int epi,
                                 uint16_t* out, void* ws, size_t ws_bytes, int32_t* dev_status,
                                 cudaStream_t stream, int sm_count);
+bool w4_tc_supported(int N, int K, int epi);
+size_t w4_tc_workspace_bytes(int64_t a_rows, int K);
+w4_status w4_launch_tc_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int k_div,
+                            const uint32_t* codes, const uint16_t* scales, const int32_t* offsets,
+                            int E, int64_t rows, int N, int K, int epi, uint16_t* out, void* ws,
+                            size_t ws_bytes, int32_t* dev_status, cudaStream_t stream, int sm_count);
+
+// Path choice: the tensor-core tile kernel when the routed rows per weight matrix make a real
+// dense contraction (on average >= 32 rows per expert, or >= 64 rows for a dense linear) and the
+// shapes fit its tiles; the weight-streaming kernel otherwise.
+static bool use_tc(int64_t rows, int E, int N, int K, int epi, bool dense, const void* scales) {
+  if (!w4_tc_supported(N, K, epi)) return false;
+  if (scales && (reinterpret_cast<uintptr_t>(scales) & 15) != 0) return false;   // bulk-copied
+  return dense ? rows >= 64 : rows >= 32LL * E;
+}
 
 namespace {
 
@@ -73,12 +88,20 @@ size_t w4_workspace_bytes(int32_t op, int64_t M_or_T, int64_t N, int64_t K, int3
   switch (op) {
     case W4_OP_LINEAR:
       if (N <= 0 || K < 32 || K % 32) return 0;
+      if (use_tc(M_or_T, 1, static_cast<int>(N), static_cast<int>(K), W4_EPI_NONE, true, nullptr))
+        return w4_tc_workspace_bytes(M_or_T, static_cast<int>(K));
       return w4_stream_workspace_bytes(M_or_T, static_cast<int>(N), static_cast<int>(K), 1,
                                        W4_EPI_NONE, true, current_sm_count());
     case W4_OP_ROUTE:
       return w4_route_workspace_bytes(static_cast<int>(M_or_T), E);
-    case W4_OP_GMM:
-      return 0;
+    case W4_OP_GMM: {
+      // the tensor-core path writes every routed row in fp16, in pair order; the streaming path
+      // needs nothing
+      if (N <= 0 || K < 32 || K % 32 || E < 1 || N > (1LL << 30) || K > (1LL << 30)) return 0;
+      const bool tc = use_tc(M_or_T, E, static_cast<int>(N), static_cast<int>(K), W4_EPI_NONE, false, nullptr) ||
+                      use_tc(M_or_T, E, static_cast<int>(N), static_cast<int>(K), W4_EPI_GELU_GATE, false, nullptr);
+      return tc ? w4_tc_workspace_bytes(M_or_T, static_cast<int>(K)) : 0;
+    }
     default:
       return 0;
   }
@@ -106,6 +129,10 @@ w4_status w4a16_linear(const uint16_t* x, const uint32_t* codes, const uint16_t*
     return W4_ERR_INVALID_ARG;
   if (workspace && !aligned(workspace, 16)) return W4_ERR_INVALID_ARG;
   if (M * N > (1LL << 40)) return W4_ERR_UNSUPPORTED;
+  if (use_tc(M, 1, static_cast<int>(N), static_cast<int>(K), W4_EPI_NONE, true, scales) && M < (1LL << 31))
+    return finish(w4_launch_tc_gemm(x, nullptr, 1, codes, scales, nullptr, 1, M, static_cast<int>(N),
+                                    static_cast<int>(K), W4_EPI_NONE, y, workspace, workspace_bytes,
+                                    nullptr, static_cast<cudaStream_t>(stream), current_sm_count()));
   return finish(w4_launch_stream_gemm(x, nullptr, 1, codes, scales, nullptr, 1, M,
                                       static_cast<int>(N), static_cast<int>(K), W4_EPI_NONE, y,
                                       workspace, workspace_bytes, nullptr,
@@ -139,6 +166,10 @@ w4_status moe_w4a16_gmm(const uint16_t* a, const int32_t* a_row_of_pair, int32_t
   if (!aligned(codes, 16) || !aligned(scales, 4) || (a && !aligned(a, 16)) || (out && !aligned(out, 16)))
     return W4_ERR_INVALID_ARG;
   if (static_cast<int64_t>(E) * N > (1LL << 31) - 1 || rows > (1LL << 31) - 1) return W4_ERR_UNSUPPORTED;
+  if (use_tc(rows, E, N, K, epilogue, false, scales))
+    return finish(w4_launch_tc_gemm(a, a_row_of_pair, k, codes, scales, expert_offsets, E, rows, N, K,
+                                    epilogue, out, workspace, workspace_bytes, dev_status,
+                                    static_cast<cudaStream_t>(stream), current_sm_count()));
   return finish(w4_launch_stream_gemm(a, a_row_of_pair, k, codes, scales, expert_offsets, E, rows, N,
                                       K, epilogue, out, workspace, workspace_bytes, dev_status,
                                       static_cast<cudaStream_t>(stream), current_sm_count()));
