@@ -172,7 +172,8 @@ def kernel_source_hash():
 
 
 def read_profile_traffic(name):
-    """dram bytes per launch from a committed ncu summary, if taken on the current kernel source."""
+    """DRAM bytes of one step's grouped-GEMM launches from a committed ncu summary, if taken on
+    the current kernel source (None otherwise)."""
     path = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(path):
         return None
@@ -184,7 +185,7 @@ def read_profile_traffic(name):
     if vals.get("kernel_source_sha256_16") != kernel_source_hash():
         return None
     try:
-        return float(vals["dram_bytes_per_launch"])
+        return float(vals["dram_bytes_per_step"])
     except (KeyError, ValueError):
         return None
 
