@@ -22,19 +22,20 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
                                 const int32_t* offsets, int E, int64_t rows, int N, int K, int epi,
                                 uint16_t* out, void* ws, size_t ws_bytes, int32_t* dev_status,
                                 cudaStream_t stream, int sm_count);
-bool w4_tc_supported(int N, int K, int epi);
-size_t w4_tc_workspace_bytes(int64_t a_rows, int K);
-w4_status w4_launch_tc_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int k_div,
+size_t w4_tc_workspace_bytes(int64_t rows, int K);
+bool w4_tm_supported(int N, int K, int epi);
+w4_status w4_launch_tm_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int k_div,
                             const uint32_t* codes, const uint16_t* scales, const int32_t* offsets,
                             int E, int64_t rows, int N, int K, int epi, uint16_t* out, void* ws,
                             size_t ws_bytes, int32_t* dev_status, cudaStream_t stream, int sm_count);
 
-// Path choice: the tensor-core tile kernel when the routed rows per weight matrix make a real
+// Path choice: the tensor-memory kernel where the routed rows per weight matrix make a real
 // dense contraction (on average >= 32 rows per expert, or >= 64 rows for a dense linear) and the
-// shapes fit its tiles; the weight-streaming kernel otherwise.
+// shapes fit its tiles (weight tiles of 128 rows, K a multiple of 64 up to 4096); the
+// weight-streaming kernel otherwise (decode batches, dense GEMVs with split-K over the SMs).
 static bool use_tc(int64_t rows, int E, int N, int K, int epi, bool dense, const void* scales) {
-  if (!w4_tc_supported(N, K, epi)) return false;
-  if (scales && (reinterpret_cast<uintptr_t>(scales) & 15) != 0) return false;   // bulk-copied
+  if (!w4_tm_supported(N, K, epi)) return false;
+  if (scales && (reinterpret_cast<uintptr_t>(scales) & 3) != 0) return false;
   return dense ? rows >= 64 : rows >= 32LL * E;
 }
 
@@ -130,7 +131,7 @@ w4_status w4a16_linear(const uint16_t* x, const uint32_t* codes, const uint16_t*
   if (workspace && !aligned(workspace, 16)) return W4_ERR_INVALID_ARG;
   if (M * N > (1LL << 40)) return W4_ERR_UNSUPPORTED;
   if (use_tc(M, 1, static_cast<int>(N), static_cast<int>(K), W4_EPI_NONE, true, scales) && M < (1LL << 31))
-    return finish(w4_launch_tc_gemm(x, nullptr, 1, codes, scales, nullptr, 1, M, static_cast<int>(N),
+    return finish(w4_launch_tm_gemm(x, nullptr, 1, codes, scales, nullptr, 1, M, static_cast<int>(N),
                                     static_cast<int>(K), W4_EPI_NONE, y, workspace, workspace_bytes,
                                     nullptr, static_cast<cudaStream_t>(stream), current_sm_count()));
   return finish(w4_launch_stream_gemm(x, nullptr, 1, codes, scales, nullptr, 1, M,
@@ -167,7 +168,7 @@ w4_status moe_w4a16_gmm(const uint16_t* a, const int32_t* a_row_of_pair, int32_t
     return W4_ERR_INVALID_ARG;
   if (static_cast<int64_t>(E) * N > (1LL << 31) - 1 || rows > (1LL << 31) - 1) return W4_ERR_UNSUPPORTED;
   if (use_tc(rows, E, N, K, epilogue, false, scales))
-    return finish(w4_launch_tc_gemm(a, a_row_of_pair, k, codes, scales, expert_offsets, E, rows, N, K,
+    return finish(w4_launch_tm_gemm(a, a_row_of_pair, k, codes, scales, expert_offsets, E, rows, N, K,
                                     epilogue, out, workspace, workspace_bytes, dev_status,
                                     static_cast<cudaStream_t>(stream), current_sm_count()));
   return finish(w4_launch_stream_gemm(a, a_row_of_pair, k, codes, scales, expert_offsets, E, rows, N,

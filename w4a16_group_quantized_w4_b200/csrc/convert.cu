@@ -1,0 +1,93 @@
+// Conversion pass in front of the tensor-core GEMMs: activations to fp16 with a power-of-two
+// exponent per row, gathered into routed-pair order.
+//
+// Method: "Repacked QAT Gemma 4 26B-A4B serves on one TPU v6e at 1.9x FP8 throughput", section
+// "What changed in vLLM's TPU backend" (activations stay 16-bit).  fp16 with a per-row exponent
+// holds every bf16 activation within 2^31 of its row's largest exactly, so the tensor-core
+// products stay the exact a * s * q.
+#include "tcgen05.cuh"
+
+namespace w4 {
+namespace cv {
+
+// One warp per output row p: the activation row it reads (row p of `a`, or row
+// a_row_of_pair[p] / k_div when rows are gathered) is scanned for its largest finite |a|, which
+// picks f so that it lands in [2^14, 2^15); row p of a16 becomes fp16(a * 2^f) and rowmul[p] = 2^-f.
+// A bf16 value of magnitude at least 2^-17 is a multiple of 2^-24 with 8 significant bits, so fp16
+// holds it exactly: every element within a factor 2^31 of the row's largest converts exactly,
+// smaller ones round to the fp16 subnormal grid.  Infinities and NaNs pass through as fp16 inf /
+// NaN.  Writing the gathered rows in pair order lets the GEMM read whole 128-row tiles by TMA.
+__global__ void __launch_bounds__(256)
+a_to_f16_kernel(const uint16_t* __restrict__ a, const int32_t* __restrict__ a_row_of_pair, int k_div,
+                int64_t a_rows, int64_t rows, int K, uint16_t* __restrict__ a16,
+                float* __restrict__ rowmul, int32_t* dev_status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t wpb = blockDim.x >> 5;
+  const int nv = K >> 3;
+  for (int64_t row = blockIdx.x * wpb + (threadIdx.x >> 5); row < rows; row += gridDim.x * wpb) {
+    int64_t srow = row;
+    if (a_row_of_pair) {
+      srow = __ldg(a_row_of_pair + row) / k_div;
+      if (srow < 0 || srow >= a_rows) {
+        if (lane == 0) set_status(dev_status, W4_ERR_INVALID_ARG);
+        srow = 0;
+      }
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(a + srow * K);
+    uint32_t m = 0;
+    for (int i = lane; i < nv; i += 32) {
+      const uint4 v = __ldg(src + i);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t lo = w[j] & 0x7FFFu, hi = (w[j] >> 16) & 0x7FFFu;
+        if (lo < 0x7F80u) m = max(m, lo);
+        if (hi < 0x7F80u) m = max(m, hi);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const int f = shift_for(m, 14);
+    const float mul = pow2f(f);
+    uint4* dst = reinterpret_cast<uint4*>(a16 + row * K);
+    for (int i = lane; i < nv; i += 32) {
+      const uint4 v = __ldg(src + i);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __half2 h = __floats2half2_rn(bf16_lo_to_f32(w[j]) * mul, bf16_hi_to_f32(w[j]) * mul);
+        o[j] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    if (lane == 0) rowmul[row] = pow2f(-f);
+  }
+}
+
+}  // namespace cv
+}  // namespace w4
+
+// fp16 activation rows in pair order [rows, K] (256-byte aligned), then the row multipliers
+size_t w4_tc_workspace_bytes(int64_t rows, int K) {
+  if (rows <= 0) return 0;
+  return (static_cast<size_t>(rows) * K * 2 + 255) / 256 * 256 + static_cast<size_t>(rows) * 4;
+}
+
+uint16_t* w4_ws_a16(void* ws) { return static_cast<uint16_t*>(ws); }
+
+float* w4_ws_rowmul(void* ws, int64_t rows, int K) {
+  return reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                  (static_cast<size_t>(rows) * K * 2 + 255) / 256 * 256);
+}
+
+void w4_launch_a_to_f16(const uint16_t* a, const int32_t* a_row_of_pair, int k_div, int64_t a_rows,
+                        int64_t rows, int K, void* ws, int32_t* dev_status, cudaStream_t stream,
+                        int sm_count) {
+  if (rows <= 0) return;
+  const int64_t blocks = (rows + 7) / 8;
+  const int grid = static_cast<int>(blocks < 16LL * sm_count ? blocks : 16LL * sm_count);
+  w4::cv::a_to_f16_kernel<<<grid, 256, 0, stream>>>(a, a_row_of_pair, k_div, a_rows, rows, K,
+                                                    w4_ws_a16(ws), w4_ws_rowmul(ws, rows, K),
+                                                    dev_status);
+}
