@@ -91,7 +91,7 @@ struct Args {
 // dequantised weights, NSPLIT x KSPLIT MMA-issuing threads (token-column parts x k parts).
 // KSK = 256 makes every code-row request of the TMA 128 bytes long; KSK = 128 leaves room for
 // 128-row token tiles.
-template <int NMAX, int KSK, int TSTAGES, int ASLOTS, int NSPLIT, int KSPLIT>
+template <int NMAX, int KSK, int TSTAGES, int ASLOTS, int NSPLIT, int KSPLIT, int ABUF, int EPIW>
 struct Cfg {
   static_assert(NMAX % 16 == 0 && NMAX <= 256, "MMA N");
   static_assert(KSK == 128 || KSK == 256, "stage width");
@@ -101,14 +101,21 @@ struct Cfg {
   static constexpr int kCodeStage = kBM * kCodePitch;
   static constexpr int kTokSub = NMAX * 128;             // one 64-k sub-tile: NMAX rows x 128 B
   static constexpr int kTokStage = kSubs * kTokSub;
+  static_assert(ABUF == 1 || ABUF == 2, "accumulator buffers");
+  static_assert(EPIW == 1 || EPIW == 2, "epilogue warps per TMEM lane quadrant");
   static constexpr int kIssuers = NSPLIT * KSPLIT;
+  static constexpr int kEpiWarps = 4 * EPIW;
+  // warps: 0-15 fixed roles, then issuers 1.., then the second epilogue warp of each quadrant
+  static constexpr int kIssuerWarp0 = 16;
+  static constexpr int kEpiWarp1 = 16 + kIssuers - 1;
+  static constexpr int kWarps = 16 + (kIssuers - 1) + 4 * (EPIW - 1);
   static constexpr int kNS = NMAX / NSPLIT;              // token columns per issuer
   static_assert(kNS % 16 == 0, "M = 128 MMAs take N in multiples of 16");
-  // accumulator (buffer ab, k part kp) at columns [(2 kp + ab) NMAX, ... + NMAX); A slots after
+  // accumulator (buffer ab, k part kp) at columns [(ABUF kp + ab) NMAX, ... + NMAX); A slots after
   __host__ __device__ static constexpr uint32_t acc_col(int ab, int kp) {
-    return static_cast<uint32_t>((2 * kp + ab) * NMAX);
+    return static_cast<uint32_t>((ABUF * kp + ab) * NMAX);
   }
-  static constexpr int kA0 = 2 * KSPLIT * NMAX;
+  static constexpr int kA0 = ABUF * KSPLIT * NMAX;
   static constexpr int kColsUsed = kA0 + ASLOTS * kACols;
   static_assert(kColsUsed <= 512, "TMEM columns");
   static constexpr uint32_t kTmemCols = kColsUsed <= 32 ? 32 : kColsUsed <= 64 ? 64
@@ -127,8 +134,11 @@ struct Tile {
   int mrows;
 };
 
-// Tile t -> (expert, block of routed rows, weight tile); m-blocks fastest, so CTAs running
-// together work on the same weight tile.
+// Tile t -> (expert, block of routed rows, weight tile); weight tiles fastest, so the CTAs
+// running together share a few token blocks (each read from HBM once and then from L2 by every
+// weight tile) while each expert's weight tiles are re-read once per token block.  (Token blocks
+// fastest would re-read every token block once per weight tile: for the prefill gate/up GEMM,
+// 1.4 MB x 11 per block, far more than the weights.)
 __device__ __forceinline__ void decode_tile(const Args& A, const int* table, const int* offs,
                                             int t, int nmax, Tile& T) {
   int lo = 0, hi = A.E - 1;
@@ -138,10 +148,9 @@ __device__ __forceinline__ void decode_tile(const Args& A, const int* table, con
   }
   T.e = lo;
   const int off0 = offs[lo], off1 = offs[lo + 1];
-  const int nm = (off1 - off0 + nmax - 1) / nmax;
   const int local = t - table[lo];
-  T.nt = local / nm;
-  T.mt = local - T.nt * nm;
+  T.mt = local / A.n_tiles;
+  T.nt = local - T.mt * A.n_tiles;
   T.r0 = off0 + static_cast<int64_t>(T.mt) * nmax;
   T.mrows = min(nmax, off1 - static_cast<int>(T.r0));
 }
@@ -193,11 +202,11 @@ __device__ __forceinline__ void scale_pair(uint32_t s16, float smul, uint32_t& s
 }
 
 
-template <int NMAX, int KSK, int TSTAGES, int ASLOTS, int NSPLIT, int KSPLIT>
-__global__ void __launch_bounds__(kThreads + 32 * (NSPLIT * KSPLIT - 1), 1)
+template <int NMAX, int KSK, int TSTAGES, int ASLOTS, int NSPLIT, int KSPLIT, int ABUF, int EPIW>
+__global__ void __launch_bounds__(32 * (16 + (NSPLIT * KSPLIT - 1) + 4 * (EPIW - 1)), 1)
 tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
                const __grid_constant__ CUtensorMap tmap_tok, Args A) {
-  using C = Cfg<NMAX, KSK, TSTAGES, ASLOTS, NSPLIT, KSPLIT>;
+  using C = Cfg<NMAX, KSK, TSTAGES, ASLOTS, NSPLIT, KSPLIT, ABUF, EPIW>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const Lay& L = A.L;
@@ -267,11 +276,11 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], C::kIssuers);
-      mbar_init(&acc_empty[b], 4);   // the epilogue warps
+      mbar_init(&acc_empty[b], C::kEpiWarps);
       mbar_init(&sc_full[b], 32);    // the scale loader's lanes (cp.async arrivals)
       mbar_init(&sc_empty[b], 8);
       mbar_init(&sh_full[b], 4);     // the dequant warps of the first k half
-      mbar_init(&sh_empty[b], 4);    // the epilogue warps
+      mbar_init(&sh_empty[b], C::kEpiWarps);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -341,7 +350,7 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       if (!ok) fail(0);
     }
     __syncwarp();
-  } else if (warp == 1 || warp >= 16) {
+  } else if (warp == 1 || (warp >= C::kIssuerWarp0 && warp < C::kEpiWarp1)) {
     // ------------------------------ MMA issuers ------------------------------
     // One thread issues tcgen05.mma at about one instruction per 86+ cycles; C::kIssuers threads
     // (lane 0 of warp 1 and of warps 16, 17, ...) share each A slot: issuer i takes the token
@@ -357,8 +366,8 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++ti) {
         Tile T;
         decode_tile(A, table, offs, t, NMAX, T);
-        const int ab = ti & 1;
-        if (ti >= 2 && !mbar_wait(&acc_empty[ab], ((ti >> 1) - 1) & 1)) { ok = false; break; }
+        const int ab = ti % ABUF, use = ti / ABUF;
+        if (ti >= ABUF && !mbar_wait(&acc_empty[ab], (use - 1) & 1)) { ok = false; break; }
         tc_fence_after();
         int n_my = ((T.mrows + 15) & ~15) - nsi * C::kNS;       // this issuer's token columns
         n_my = n_my < 0 ? 0 : (n_my > C::kNS ? C::kNS : n_my);
@@ -420,25 +429,28 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
                    : "memory");
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
-  } else if (warp >= 4 && warp < 8) {
+  } else if ((warp >= 4 && warp < 8) || warp >= C::kEpiWarp1) {
     // ------------------------------ epilogue ------------------------------
-    const int q = warp - 4;                     // TMEM lanes 32q .. 32q + 31
+    // TMEM lanes 32q .. 32q+31 are readable by warps with warp % 4 == q; with two epilogue warps
+    // per quadrant, part cp takes the 16-column chunks cp, cp + 2, ...
+    const int q = warp & 3;
+    const int cp = warp < 8 ? 0 : 1;
     const int l = q * 32 + lane;
     const bool gelu = A.epi == W4_EPI_GELU_GATE;
     int ti = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++ti) {
       Tile T;
       decode_tile(A, table, offs, t, NMAX, T);
-      const int ab = ti & 1;
-      if (!mbar_wait(&acc_full[ab], (ti >> 1) & 1)) { fail(lane); break; }
+      const int ab = ti % ABUF, hb = ti & 1;
+      if (!mbar_wait(&acc_full[ab], (ti / ABUF) & 1)) { fail(lane); break; }
       tc_fence_after();
-      if (!mbar_wait(&sh_full[ab], (ti >> 1) & 1)) { fail(lane); break; }
-      const float cm = sh[ab * kBM + l];          // 2^-e of this lane's weight row
+      if (!mbar_wait(&sh_full[hb], (ti >> 1) & 1)) { fail(lane); break; }
+      const float cm = sh[hb * kBM + l];          // 2^-e of this lane's weight row
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh_empty[ab]);
+      if (lane == 0) mbar_arrive(&sh_empty[hb]);
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       const int n_cols = (T.mrows + 15) & ~15;
-      for (int c0 = 0; c0 < n_cols; c0 += 16) {
+      for (int c0 = 16 * cp; c0 < n_cols; c0 += 16 * EPIW) {
         float v[16];
         tmem_ld16(taddr + C::acc_col(ab, 0) + c0, v);
 #pragma unroll
@@ -607,9 +619,9 @@ bool w4_tm_supported(int N, int K, int epi) {
 // shared memory of one CTA (the opt-in maximum minus the 1024-byte alignment slack)
 constexpr int kTmSmemBudget = 232448 - 1024;
 
-template <int NMAX, int KSK, int TSTAGES, int ASLOTS, int NSPLIT, int KSPLIT>
+template <int NMAX, int KSK, int TSTAGES, int ASLOTS, int NSPLIT, int KSPLIT, int ABUF, int EPIW>
 static bool tm_layout(int E, int kg, w4::tm::Lay& L) {
-  using C = w4::tm::Cfg<NMAX, KSK, TSTAGES, ASLOTS, NSPLIT, KSPLIT>;
+  using C = w4::tm::Cfg<NMAX, KSK, TSTAGES, ASLOTS, NSPLIT, KSPLIT, ABUF, EPIW>;
   L.code = C::code;
   L.scb = (w4::tm::kBM * ((kg >> 1) | 1) * 4 + 127) / 128 * 128;
   const int fixed = 2 * L.scb + 2 * w4::tm::kBM * 4 + C::nbars * 8 + 16 + (E + 1) * 8;
@@ -626,13 +638,13 @@ static bool tm_layout(int E, int kg, w4::tm::Lay& L) {
   return L.total <= kTmSmemBudget;
 }
 
-template <int NMAX, int KSK, int TSTAGES, int ASLOTS, int NSPLIT, int KSPLIT>
+template <int NMAX, int KSK, int TSTAGES, int ASLOTS, int NSPLIT, int KSPLIT, int ABUF, int EPIW>
 static w4_status tm_launch_cfg(const uint32_t* codes, const uint16_t* a16, int64_t rows, int K,
                                w4::tm::Args A, cudaStream_t stream, int sm_count) {
-  using C = w4::tm::Cfg<NMAX, KSK, TSTAGES, ASLOTS, NSPLIT, KSPLIT>;
+  using C = w4::tm::Cfg<NMAX, KSK, TSTAGES, ASLOTS, NSPLIT, KSPLIT, ABUF, EPIW>;
   auto fn = tm_encode_fn();
   if (!fn) return W4_ERR_CUDA;
-  if (!tm_layout<NMAX, KSK, TSTAGES, ASLOTS, NSPLIT, KSPLIT>(A.E, A.kg, A.L)) return W4_ERR_UNSUPPORTED;
+  if (!tm_layout<NMAX, KSK, TSTAGES, ASLOTS, NSPLIT, KSPLIT, ABUF, EPIW>(A.E, A.kg, A.L)) return W4_ERR_UNSUPPORTED;
   A.nst = (K + KSK - 1) / KSK;
   cuuint32_t estr[2] = {1, 1};
   // raw codes [E*N, K/8] words: box = one stage of k (KSK/8 words) x 64 rows, swizzled to the
@@ -664,13 +676,13 @@ static w4_status tm_launch_cfg(const uint32_t* codes, const uint16_t* a16, int64
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(w4::tm::tm_gemm_kernel<NMAX, KSK, TSTAGES, ASLOTS, NSPLIT, KSPLIT>,
+    if (cudaFuncSetAttribute(w4::tm::tm_gemm_kernel<NMAX, KSK, TSTAGES, ASLOTS, NSPLIT, KSPLIT, ABUF, EPIW>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 232448) != cudaSuccess)
       return W4_ERR_CUDA;
     attr_done[dev] = 1;
   }
-  w4::tm::tm_gemm_kernel<NMAX, KSK, TSTAGES, ASLOTS, NSPLIT, KSPLIT>
-      <<<sm_count, w4::tm::kThreads + 32 * (C::kIssuers - 1), smem, stream>>>(tmap_codes, tmap_tok, A);
+  w4::tm::tm_gemm_kernel<NMAX, KSK, TSTAGES, ASLOTS, NSPLIT, KSPLIT, ABUF, EPIW>
+      <<<sm_count, 32 * C::kWarps, smem, stream>>>(tmap_codes, tmap_tok, A);
   return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
@@ -697,6 +709,8 @@ w4_status w4_launch_tm_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int
   A.n_tiles = (epi == W4_EPI_GELU_GATE) ? (N / 2) / (w4::tm::kBM / 2) : N / w4::tm::kBM;
   A.dev_status = dev_status;
   const uint16_t* a16 = w4_ws_a16(ws);
-  // 128-row token blocks, 128-k stages, one MMA-issuing thread
-  return tm_launch_cfg<128, 128, 3, 2, 1, 1>(codes, a16, rows, K, A, stream, sm_count);
+  // 256-row token blocks, 128-k stages, two MMA-issuing threads (128 token columns each, the
+  // tensor pipe's rate needs more than one issuer), one 256-column accumulator drained by eight
+  // epilogue warps
+  return tm_launch_cfg<192, 128, 2, 2, 2, 1, 2, 2>(codes, a16, rows, K, A, stream, sm_count);
 }
