@@ -1,0 +1,116 @@
+"""Repack + full expert stack: 30 layers x 128 experts of planted bf16 weights, recovered on the
+device (bit-exact against the planted codes and the oracle's scales, zero groups off the grid),
+then decode through all 30 layers at 1, 32 and 256 tokens.
+
+Definition: "Repacked QAT Gemma 4 26B-A4B serves on one TPU v6e at 1.9x FP8 throughput", section
+"A repack, not a re-quantization" (every group sits on the -8..7 grid; the repack searches
+max|w|/m, refines by least squares and packs; verification found zero groups off the grid) and
+"The gap at 26B" (128 experts per layer, 8 active).  Planted groups: peak level uniform in 1..8,
+scales log-uniform in [1e-4, 1e-1] at binade resolution (synth.planted_groups).  The device
+generator is checked bit for bit against the host one first.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe, q4
+from w4a16_group_quantized_w4_b200 import stack, synth, synth_device
+from tests._util import assert_rows_close, dev_bf16, dev_f32, host_f64
+
+pytestmark = pytest.mark.gpu
+
+L, E, K_TOP, H, I = 30, 128, 8, 2816, 704
+GU_STREAM, DN_STREAM = 500, 501
+
+
+def _host_bits(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def test_device_generator_matches_host():
+    n = 257
+    for stream, g0 in ((GU_STREAM, 0), (GU_STREAM, 123_456_789), (DN_STREAM, L * E * H * I // 32 - n)):
+        w, q, s = synth_device.planted(n, g0, 0, stream, with_truth=True)
+        ref = synth.planted_groups(np.arange(g0, g0 + n), 0, stream)
+        assert np.array_equal(_host_bits(w).reshape(n, 32), ref.w)
+        assert np.array_equal(q.cpu().numpy(), ref.q)
+        assert np.array_equal(_host_bits(s), ref.s)
+
+
+@pytest.fixture(scope="module")
+def c5():
+    st = stack.MoEStack(L, E, K_TOP, H, I)
+    n_gu = st.gate_up_rows() * H // 32
+    n_dn = st.down_rows() * I // 32
+    w_gu = synth_device.planted(n_gu, 0, 0, GU_STREAM).view(st.gate_up_rows(), H)
+    w_dn = synth_device.planted(n_dn, 0, 0, DN_STREAM).view(st.down_rows(), I)
+    rep = st.repack(w_gu, w_dn)
+    torch.cuda.synchronize()
+    del w_gu, w_dn
+    torch.cuda.empty_cache()
+    yield st, rep, n_gu, n_dn
+    del st, rep
+    torch.cuda.empty_cache()
+
+
+def test_repack_full_stack_codes_match_planted(c5):
+    st, rep, n_gu, n_dn = c5
+    assert rep.off_grid_gate_up == 0 and rep.off_grid_down == 0
+    assert synth_device.code_mismatches(st.gu_codes.view(-1), 0, n_gu, 0, GU_STREAM) == 0
+    assert synth_device.code_mismatches(st.dn_codes.view(-1), 0, n_dn, 0, DN_STREAM) == 0
+
+
+@pytest.mark.parametrize("which,layer,expert", [("gu", 0, 0), ("gu", 29, 127), ("dn", 0, 5), ("dn", 29, 127)])
+def test_repack_sampled_rows_match_oracle(c5, which, layer, expert):
+    """64 rows of one expert: codes, scales and group_m bit-exact against the oracle's repack of
+    the host-generated planted weights; group_m equals the planted peak level."""
+    st, rep, _, _ = c5
+    if which == "gu":
+        K, stream, per = H, GU_STREAM, 2 * I
+        codes, scales, gm = st.gu_codes.view(-1, H // 8), st.gu_scales.view(-1, H // 32), rep.group_m_gate_up
+    else:
+        K, stream, per = I, DN_STREAM, H
+        codes, scales, gm = st.dn_codes.view(-1, I // 8), st.dn_scales.view(-1, I // 32), rep.group_m_down
+    row0 = (layer * E + expert) * per + per - 64
+    pg = synth.planted_weights(64, K, 0, stream, row0=row0)
+    ref = q4.repack(pg.w.reshape(64, K))
+    assert ref.off_grid == 0
+    assert np.array_equal(codes[row0:row0 + 64].cpu().numpy().view(np.uint32), ref.codes)
+    assert np.array_equal(_host_bits(scales[row0:row0 + 64]), ref.scales)
+    assert np.array_equal(gm[row0:row0 + 64].cpu().numpy(), ref.group_m)
+    assert np.array_equal(ref.group_m.ravel(), pg.peak.astype(np.uint8))
+
+
+def _oracle_layer_for_tokens(layer, x, logits, tokens):
+    """The oracle's MoE layer for the given tokens, with the weights of every expert those tokens
+    route to generated on the host and repacked by the oracle (other experts stay zero)."""
+    rt = moe.route(logits, K_TOP)
+    hit = np.unique(rt.topk_ids[tokens])
+    gu_c = np.zeros((E, 2 * I, H // 8), np.uint32)
+    gu_s = np.zeros((E, 2 * I, H // 32), np.uint16)
+    dn_c = np.zeros((E, H, I // 8), np.uint32)
+    dn_s = np.zeros((E, H, I // 32), np.uint16)
+    for e in hit:
+        e = int(e)
+        g = synth.planted_weights(2 * I, H, 0, GU_STREAM, row0=(layer * E + e) * 2 * I)
+        r = q4.repack(g.w.reshape(2 * I, H))
+        gu_c[e], gu_s[e] = r.codes, r.scales
+        d = synth.planted_weights(H, I, 0, DN_STREAM, row0=(layer * E + e) * H)
+        r = q4.repack(d.w.reshape(H, I))
+        dn_c[e], dn_s[e] = r.codes, r.scales
+    return moe.moe_layer(x, logits, gu_c, gu_s, dn_c, dn_s, K_TOP, tokens=tokens)
+
+
+@pytest.mark.parametrize("T,layer,tokens", [(1, 0, [0]), (1, 29, [0]), (32, 15, [5]), (256, 29, [255])])
+def test_decode_through_stack_matches_oracle(c5, T, layer, tokens):
+    """One decode step through all 30 layers at T tokens; the sampled tokens of one layer against
+    the oracle (each layer has its own seeded inputs and router logits)."""
+    st = c5[0]
+    xs = [synth.bf16_normal((T, H), 0, 600 + l) for l in range(L)]
+    lgs = [synth.router_logits(T, E, 0, 700 + l) for l in range(L)]
+    ys = st.step([dev_bf16(x) for x in xs], [dev_f32(g) for g in lgs])
+    torch.cuda.synchronize()
+    for y in ys:
+        assert torch.isfinite(y.float()).all()
+    ref = _oracle_layer_for_tokens(layer, xs[layer], lgs[layer], np.asarray(tokens))
+    assert_rows_close(host_f64(ys[layer])[tokens], ref.y[tokens])

@@ -1,0 +1,84 @@
+"""A stack of mixture-of-experts layers held on one device.
+
+The whole-model form of the hot path: every layer's gate/up and down weights arrive as bf16 (the
+"unquantized" QAT export of "Repacked QAT Gemma 4 26B-A4B serves on one TPU v6e at 1.9x FP8
+throughput", section "A repack, not a re-quantization"), are repacked on the device by
+`w4_repack` into int4 codes and bf16 scales, and decode steps then run the four entry points layer
+after layer ("The gap at 26B": 128 experts per layer, 8 active).  The pages give no blocks
+between the MoE layers, so each layer takes its own input rows and router logits.
+
+Layouts (layer-major, so layer l's weights are contiguous slices):
+  gate/up codes [L, E, 2I, H/8] int32, scales [L, E, 2I, H/32] bf16
+  down    codes [L, E, H, I/8]  int32, scales [L, E, H, I/32]  bf16
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import api
+
+
+@dataclass
+class RepackReport:
+    off_grid_gate_up: int
+    off_grid_down: int
+    group_m_gate_up: torch.Tensor     # uint8 [L*E*2I, H/32]
+    group_m_down: torch.Tensor        # uint8 [L*E*H, I/32]
+
+
+class MoEStack:
+    """L layers of E experts (hidden H, expert intermediate I, top-k routing) on one device."""
+
+    def __init__(self, L: int, E: int = 128, k: int = 8, H: int = 2816, I: int = 704, device="cuda"):
+        self.L, self.E, self.k, self.H, self.I = L, E, k, H, I
+        dev = torch.device(device)
+        self.gu_codes = torch.empty((L, E, 2 * I, H // 8), dtype=torch.int32, device=dev)
+        self.gu_scales = torch.empty((L, E, 2 * I, H // 32), dtype=torch.bfloat16, device=dev)
+        self.dn_codes = torch.empty((L, E, H, I // 8), dtype=torch.int32, device=dev)
+        self.dn_scales = torch.empty((L, E, H, I // 32), dtype=torch.bfloat16, device=dev)
+        self._layers = {}
+
+    # ------------------------------------------------------------------ repack
+    def gate_up_rows(self) -> int:
+        return self.L * self.E * 2 * self.I
+
+    def down_rows(self) -> int:
+        return self.L * self.E * self.H
+
+    def repack(self, w_gate_up: torch.Tensor, w_down: torch.Tensor, stream=None) -> RepackReport:
+        """w_gate_up bf16 [L*E*2I, H], w_down bf16 [L*E*H, I] (layer-major) -> this stack's codes
+        and scales, through two w4_repack calls."""
+        dev = self.gu_codes.device
+        g_gu = torch.empty((self.gate_up_rows(), self.H // 32), dtype=torch.uint8, device=dev)
+        g_dn = torch.empty((self.down_rows(), self.I // 32), dtype=torch.uint8, device=dev)
+        off = torch.zeros(2, dtype=torch.int64, device=dev)
+        api.w4_repack(w_gate_up, codes=self.gu_codes.view(-1, self.H // 8),
+                      scales=self.gu_scales.view(-1, self.H // 32), group_m=g_gu,
+                      off_grid_count=off[0:1], stream=stream)
+        api.w4_repack(w_down, codes=self.dn_codes.view(-1, self.I // 8),
+                      scales=self.dn_scales.view(-1, self.I // 32), group_m=g_dn,
+                      off_grid_count=off[1:2], stream=stream)
+        o = off.cpu()
+        return RepackReport(int(o[0]), int(o[1]), g_gu, g_dn)
+
+    # ------------------------------------------------------------------ decode
+    def layer(self, l: int, T: int) -> api.MoELayer:
+        """The four-call MoE layer l for T tokens (buffers allocated once per (l, T))."""
+        key = (l, T)
+        if key not in self._layers:
+            self._layers[key] = api.MoELayer(self.gu_codes[l], self.gu_scales[l], self.dn_codes[l],
+                                             self.dn_scales[l], T, self.k)
+        return self._layers[key]
+
+    def step(self, xs, logits, stream=None):
+        """One decode step through every layer: xs[l] bf16 [T, H], logits[l] f32 [T, E] -> the
+        list of layer outputs y_l bf16 [T, H] (each layer's own buffer)."""
+        T = xs[0].shape[0]
+        return [self.layer(l, T)(xs[l], logits[l], stream=stream) for l in range(self.L)]
+
+    def expert_bytes(self) -> int:
+        """Packed bytes of one expert (gate/up + down codes and scales)."""
+        return (2 * self.I * self.H // 2 + 2 * self.I * self.H // 16 +
+                self.H * self.I // 2 + self.H * self.I // 16)
