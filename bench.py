@@ -463,7 +463,67 @@ def run_secondary(args, device, stream):
                                             "frac_bf16_peak": round(flops / ms / 1e9 / tc_peak, 3)}
         del lay
         torch.cuda.empty_cache()
+    out.update(run_stack(device, stream))
     return out
+
+
+def run_stack(device, stream, L=30, reps=3):
+    """Repack + full expert stack: 30 layers x 128 experts of planted bf16 weights (generated on
+    the device), repacked, then decode steps through all 30 layers at 1, 32 and 256 tokens."""
+    import torch
+
+    from w4a16_group_quantized_w4_b200 import stack, synth, synth_device
+    res = {}
+    hbm_peak, _, _, _ = peaks()
+    st = stack.MoEStack(L)
+    H, I, E = st.H, st.I, st.E
+    w_gu = synth_device.planted(st.gate_up_rows() * H // 32, 0, 0, 500).view(st.gate_up_rows(), H)
+    w_dn = synth_device.planted(st.down_rows() * I // 32, 0, 0, 501).view(st.down_rows(), I)
+    with torch.cuda.stream(stream):
+        rep = st.repack(w_gu, w_dn, stream=stream)          # warm-up (also the parity-checked result)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            st.repack(w_gu, w_dn, stream=stream)
+        e1.record(stream)
+    stream.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    groups = (st.gate_up_rows() * H + st.down_rows() * I) // 32
+    moved = groups * (64 + 16 + 2 + 1)          # bf16 in; codes, scale, group_m out
+    res["repack_30x128_experts"] = {"ms": round(ms, 3), "groups": groups, "GB/s": round(moved / ms / 1e6, 1),
+                                    "frac_hbm": round(moved / ms / 1e6 / hbm_peak, 3),
+                                    "off_grid": rep.off_grid_gate_up + rep.off_grid_down}
+    del w_gu, w_dn, rep
+    torch.cuda.empty_cache()
+    for T in (1, 32, 256):
+        xs = [to_dev(synth.bf16_normal((T, H), 0, 600 + l), "bf16", device) for l in range(L)]
+        lgs = [to_dev(synth.router_logits(T, E, 0, 700 + l), "f32", device) for l in range(L)]
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                st.step(xs, lgs, stream=stream)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                st.step(xs, lgs, stream=stream)
+            g.replay()
+        stream.synchronize()
+        hit = sum(int((torch.diff(st.layer(l, T).rt.expert_offsets) > 0).sum()) for l in range(L))
+        n = 20
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(n):
+                g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        ms = e0.elapsed_time(e1) / n
+        byts = hit * st.expert_bytes() + L * T * H * 2 * 2
+        res[f"stack_decode_30_layers_T{T}"] = {"ms_per_step": round(ms, 3), "tokens/s": round(T / ms * 1e3, 1),
+                                               "experts_hit": hit, "GB/s": round(byts / ms / 1e6, 1),
+                                               "frac_hbm": round(byts / ms / 1e6 / hbm_peak, 3)}
+        del g
+    del st
+    torch.cuda.empty_cache()
+    return res
 
 
 # ------------------------------------------------------------------------------------------
