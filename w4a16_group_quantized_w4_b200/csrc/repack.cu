@@ -6,7 +6,7 @@
 // The exact rule (float64, tolerance 1/16, off-grid fallback, zero and non-finite groups) is the
 // one stated beside w4_repack in w4a16.h; results are bit-identical to it.
 //
-// Work mapping: one thread per group (64 input bytes -> 16 code bytes, 2 scale bytes, 1 m byte),
+// Work mapping: four lanes per group (64 input bytes -> 16 code bytes, 2 scale bytes, 1 m byte),
 // grid-stride over all groups.  HBM-bound when the ALU work per group stays small, so the
 // m-search runs in float32 with a guard band and only falls back to the exact float64 search
 // when the float32 evidence cannot decide:
@@ -48,126 +48,221 @@ struct GroupBits {
 };
 
 __device__ __forceinline__ float elem_f32(const GroupBits& g, int i) {
-  return (i & 1) ? bf16_hi_to_f32(g.v[i >> 1]) : bf16_lo_to_f32(g.v[i >> 1]);
+  return (i & 1) ? bf16_lo_to_f32(g.v[i >> 1] >> 16) : bf16_lo_to_f32(g.v[i >> 1]);
 }
 
-// Exact float64 search and off-grid fallback, the rule's own arithmetic.
-__device__ __forceinline__ int search_exact(const GroupBits& g, double a, int (&q)[32]) {
+// Bit position of element i's nibble inside code word i / 8 (layout L1: even elements in the low
+// half-word, odd ones in the high half-word, two consecutive k per extracted pair).
+__host__ __device__ constexpr int nibble_shift(int i) { return 4 * ((i & 7) >> 1) + 16 * (i & 1); }
+
+__device__ __forceinline__ int code_of(const uint32_t (&cw)[4], int i) {
+  return static_cast<int>((cw[i >> 3] >> nibble_shift(i)) & 15u) - 8;
+}
+
+// Exact float64 search and off-grid fallback, the rule's own arithmetic (rarely taken).
+__device__ __noinline__ int search_exact(const GroupBits& g, double a, uint32_t (&cw)[4]) {
   for (int m = 1; m <= 8; ++m) {
     const double step = a / static_cast<double>(m);
     bool ok = true;
+    uint32_t t[4] = {0, 0, 0, 0};
     for (int i = 0; i < 32; ++i) {
       const double r = static_cast<double>(elem_f32(g, i)) / step;
       const double qi = rint(r);
       if (fabs(r - qi) > 0.0625 || qi < -8.0 || qi > 7.0) { ok = false; break; }
-      q[i] = static_cast<int>(qi);
+      t[i >> 3] |= static_cast<uint32_t>(static_cast<int>(qi) + 8) << nibble_shift(i);
     }
-    if (ok) return m;
+    if (ok) {
+      for (int j = 0; j < 4; ++j) cw[j] = t[j];
+      return m;
+    }
   }
   const double step8 = a / 8.0;
+  uint32_t t[4] = {0, 0, 0, 0};
   for (int i = 0; i < 32; ++i) {
     double qi = rint(static_cast<double>(elem_f32(g, i)) / step8);
     qi = fmin(fmax(qi, -8.0), 7.0);
-    q[i] = static_cast<int>(qi);
+    t[i >> 3] |= static_cast<uint32_t>(static_cast<int>(qi) + 8) << nibble_shift(i);
   }
+  for (int j = 0; j < 4; ++j) cw[j] = t[j];
   return 0;
 }
 
-// float32 guard-band search.  Returns m in 1..8 when decided (codes in q), 0 when the exact
-// path must decide.
-__device__ __forceinline__ int search_fast(const GroupBits& g, float a, int (&q)[32]) {
-  const float tol = 0.0625f, band = 0x1p-17f;
-  const float ra = __frcp_rn(a);
-#pragma unroll 1
-  for (int m = 1; m <= 8; ++m) {
-    const float inv = __fmul_rn(static_cast<float>(m), ra);
-    bool fail = false, unsure = false;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float r = __fmul_rn(elem_f32(g, i), inv);
-      const float qf = rintf(r);
-      const float d = fabsf(__fsub_rn(r, qf));
-      fail |= (d > tol + band) | (qf > 7.0f) | (qf < -8.0f);
-      unsure |= (d > tol - band);
-      q[i] = static_cast<int>(qf);
-    }
-    if (fail) continue;
-    if (unsure) return 0;
-    return m;
-  }
-  return 0;  // off the grid: decided exactly
+// Work mapping: four consecutive lanes (a quad) per group; lane `sub` of the quad holds elements
+// 8 sub .. 8 sub + 7 (one 16-byte load) and produces code word `sub`.  Decisions that involve the
+// whole group (largest magnitude, pass / fail of a step, the least-squares sums) combine the four
+// lanes with shuffles inside the quad.
+__device__ __forceinline__ uint32_t quad_max(uint32_t v, unsigned qm) {
+  v = max(v, __shfl_xor_sync(qm, v, 1));
+  return max(v, __shfl_xor_sync(qm, v, 2));
+}
+__device__ __forceinline__ uint32_t quad_min(uint32_t v, unsigned qm) {
+  v = min(v, __shfl_xor_sync(qm, v, 1));
+  return min(v, __shfl_xor_sync(qm, v, 2));
+}
+__device__ __forceinline__ uint32_t quad_or(uint32_t v, unsigned qm) {
+  v |= __shfl_xor_sync(qm, v, 1);
+  return v | __shfl_xor_sync(qm, v, 2);
 }
 
-__global__ void __launch_bounds__(256) repack_kernel(const uint4* __restrict__ w, int64_t groups,
-                                                     uint4* __restrict__ codes,
+// float32 guard-band search over this lane's 8 elements (v: element 2j in the low half of v[j]),
+// decided for the quad.  Returns m in 1..8 (this lane's code word in cw), or 0 when the exact
+// path must decide.  An m for which the smallest nonzero |w| maps to r strictly inside
+// (1/16, 15/16) cannot reproduce the group (that element is more than 1/16 from every integer),
+// so it is skipped without looking at the elements (margins of 2^-16 cover the float32 error of
+// m * wmin / a); on the grid this makes the group's own m the first candidate.  The search runs
+// in rounds over the whole warp: each round every undecided group tries its next candidate, so
+// the eight groups of a warp share one pass instead of one pass per distinct m.
+__device__ __forceinline__ int search_fast_quad(const uint32_t (&v)[4], float a, float wmin,
+                                                unsigned qm, uint32_t& cw, float& psum, float& qsum) {
+  const float tol = 0.0625f, band = 0x1p-17f, kRound = 12582912.0f;
+  const float ra = __frcp_rn(a);
+  const float rmin1 = __fmul_rn(wmin, ra);
+  auto skip = [&](int m) {
+    const float rmin = static_cast<float>(m) * rmin1;
+    return rmin > 0.0625f + 0x1p-16f && rmin < 0.9375f - 0x1p-16f;
+  };
+  int next = 1;
+  while (next <= 8 && skip(next)) ++next;
+  bool done = next > 8;                      // no candidate at all: off the grid
+  int result = 0;
+  const unsigned active = __activemask();
+  while (__any_sync(active, !done)) {
+    const float inv = __fmul_rn(static_cast<float>(next <= 8 ? next : 8), ra);
+    uint32_t t = 0, ubits = 0;
+    float dmax = 0.f, ps = 0.f, qs = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float x = (i & 1) ? __uint_as_float(v[i >> 1] & 0xFFFF0000u) : __uint_as_float(v[i >> 1] << 16);
+      const float r = __fmul_rn(x, inv);
+      // |r| <= 8 here: adding 1.5 * 2^23 rounds r to an integer n (nearest, ties to even, as
+      // rint) and leaves 2^22 + n in the fraction bits, so u = n + 8 is (bits + 8) mod 2^23
+      const float tr = __fadd_rn(r, kRound);
+      const float qf = __fsub_rn(tr, kRound);
+      const uint32_t u = __float_as_uint(tr) + 8u - 0x4B400000u;
+      dmax = fmaxf(dmax, fabsf(__fsub_rn(r, qf)));
+      ubits |= u;                                  // u = 16 (n = +8) is the only way out of range
+      t |= (u & 15u) << nibble_shift(i);
+      // least-squares sums of this candidate (exact: see the caller)
+      ps = __fmaf_rn(x, qf, ps);
+      qs = __fmaf_rn(qf, qf, qs);
+    }
+    uint32_t fail = (dmax > tol + band) | ((ubits & ~15u) != 0);
+    uint32_t unsure = dmax > tol - band;
+    fail = quad_or(fail, qm);
+    unsure = quad_or(unsure, qm);
+    if (!done) {
+      if (!fail) {
+        done = true;
+        if (!unsure) { result = next; cw = t; psum = ps; qsum = qs; }   // else 0: exact path
+      } else {
+        ++next;
+        while (next <= 8 && skip(next)) ++next;
+        done = next > 8;                               // off the grid: decided exactly
+      }
+    }
+  }
+  return result;
+}
+
+// The exact rule (and the off-grid fallback) for a quad's group, run by the quad's first lane on
+// the whole group, with the float64 sum in index order; results broadcast to the quad.  Kept out
+// of line so that the common path's register budget stays small.
+__device__ __noinline__ void exact_quad(const uint32_t (&v)[4], float a, unsigned qm, int qbase,
+                                        int sub, int& m, double& num, int& den, uint32_t& cw) {
+  GroupBits G;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) G.v[4 * k + j] = __shfl_sync(qm, v[j], qbase + k);
+  uint32_t cws[4] = {0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u};
+  int mm = 0, dd = 0;
+  double nn = 0.0;
+  if (sub == 0) {
+    mm = search_exact(G, static_cast<double>(a), cws);
+    for (int i = 0; i < 32; ++i) {
+      const int qi = code_of(cws, i);
+      nn = __fma_rn(static_cast<double>(elem_f32(G, i)), static_cast<double>(qi), nn);
+      dd += qi * qi;
+    }
+  }
+  m = __shfl_sync(qm, mm, qbase);
+  num = __shfl_sync(qm, nn, qbase);
+  den = __shfl_sync(qm, dd, qbase);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t c = __shfl_sync(qm, cws[k], qbase);
+    if (sub == k) cw = c;
+  }
+}
+
+__global__ void __launch_bounds__(256, 4) repack_kernel(const uint4* __restrict__ w, int64_t groups,
+                                                     uint32_t* __restrict__ codes,
                                                      uint16_t* __restrict__ scales,
                                                      uint8_t* __restrict__ group_m,
                                                      unsigned long long* off_grid_count) {
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t gi = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; gi < groups;
+  const int lane = threadIdx.x & 31, sub = lane & 3, qbase = lane & ~3;
+  const unsigned qm = 0xFu << qbase;
+  const int64_t stride = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 2;
+  for (int64_t gi = ((static_cast<int64_t>(blockIdx.x) * blockDim.x) + threadIdx.x) >> 2; gi < groups;
        gi += stride) {
-    GroupBits g;
+    const uint4 u = ldg_stream128(w + gi * 4 + sub);
+    const uint32_t v[4] = {u.x, u.y, u.z, u.w};
+    uint32_t amax = 0, amin = 0x7FFFu, nonfinite = 0;     // largest and smallest nonzero |w|
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint4 u = ldg_stream128(w + gi * 4 + c);
-      g.v[4 * c + 0] = u.x; g.v[4 * c + 1] = u.y; g.v[4 * c + 2] = u.z; g.v[4 * c + 3] = u.w;
-    }
-    uint32_t amax = 0, nonfinite = 0;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const uint32_t lo = g.v[i] & 0x7FFFu, hi = (g.v[i] >> 16) & 0x7FFFu;
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t lo = v[j] & 0x7FFFu, hi = (v[j] >> 16) & 0x7FFFu;
       amax = max(amax, max(lo, hi));
+      amin = min(amin, min(lo ? lo : 0x7FFFu, hi ? hi : 0x7FFFu));
       nonfinite |= ((lo & 0x7F80u) == 0x7F80u) | ((hi & 0x7F80u) == 0x7F80u);
     }
-    int q[32];
+    amax = quad_max(amax, qm);
+    amin = quad_min(amin, qm);
+    nonfinite = quad_or(nonfinite, qm);
+    uint32_t cw = 0x88888888u;                            // q = 0
     int m;
     uint16_t scale_bits;
     bool off = false;
     if (nonfinite) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) q[i] = 0;
       m = 0;
       scale_bits = 0x7FC0;
       off = true;
     } else if (amax == 0) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) q[i] = 0;
       m = 1;
       scale_bits = 0;
     } else {
       const float a = bf16_lo_to_f32(amax);
       m = 0;
-      if (a >= 0x1p-100f && a <= 0x1p100f) m = search_fast(g, a, q);
-      if (m == 0) m = search_exact(g, static_cast<double>(a), q);
-      off = (m == 0);
-      // least squares with the codes fixed: s* = sum w q / sum q^2, index order, float64
+      float ps = 0.f, qs = 0.f;
+      if (a >= 0x1p-100f && a <= 0x1p100f) m = search_fast_quad(v, a, bf16_lo_to_f32(amin), qm, cw, ps, qs);
       double num = 0.0;
       int den = 0;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        num = __dadd_rn(num, __dmul_rn(static_cast<double>(elem_f32(g, i)), static_cast<double>(q[i])));
-        den += q[i] * q[i];
+      if (m > 0) {
+        // On the grid every nonzero product w q lies within a factor 70 of the others and carries
+        // at most 12 significant bits, so sums of them are exact in any order: a lane's eight in
+        // float32 (at most about 21 bits wide), the quad's four partial sums in float64.  This is
+        // the float64 index-order sum of the rule, bit for bit.  sum q^2 <= 2048 is exact too.
+        num = static_cast<double>(ps);
+        num = __dadd_rn(num, __shfl_xor_sync(qm, num, 1));
+        num = __dadd_rn(num, __shfl_xor_sync(qm, num, 2));
+        den = static_cast<int>(qs);
+        den += __shfl_xor_sync(qm, den, 1);
+        den += __shfl_xor_sync(qm, den, 2);
+      } else {
+        exact_quad(v, a, qm, qbase, sub, m, num, den, cw);
+        off = (m == 0);
       }
       const double s = den > 0 ? __ddiv_rn(num, static_cast<double>(den)) : 0.0;
       scale_bits = f64_to_bf16_rne(s);
     }
-    uint4 packed;
-    uint32_t* pw = reinterpret_cast<uint32_t*>(&packed);
-#pragma unroll
-    for (int wd = 0; wd < 4; ++wd) {
-      uint32_t word = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j)   // even elements in the low half-word, odd in the high
-        word |= static_cast<uint32_t>(q[8 * wd + j] + 8) << (4 * (j >> 1) + 16 * (j & 1));
-      pw[wd] = word;
+    codes[gi * 4 + sub] = cw;
+    if (sub == 0) {
+      scales[gi] = scale_bits;
+      if (group_m) group_m[gi] = static_cast<uint8_t>(m);
     }
-    codes[gi] = packed;
-    scales[gi] = scale_bits;
-    if (group_m) group_m[gi] = static_cast<uint8_t>(m);
     if (off_grid_count) {
-      const unsigned ballot = __ballot_sync(__activemask(), off);
-      const int lane = threadIdx.x & 31;
-      if (ballot && lane == __ffs(__activemask()) - 1)
+      const unsigned active = __activemask();
+      const unsigned ballot = __ballot_sync(active, off && sub == 0);
+      if (ballot && lane == __ffs(active) - 1)
         atomicAdd(off_grid_count, static_cast<unsigned long long>(__popc(ballot)));
     }
   }
@@ -184,12 +279,11 @@ w4_status w4_launch_repack(const uint16_t* w, int64_t groups, uint32_t* codes, u
       return W4_ERR_CUDA;
   }
   if (groups == 0) return W4_OK;
-  const int threads = 256;
-  int64_t blocks = (groups + threads - 1) / threads;
-  const int64_t cap = static_cast<int64_t>(sm_count) * 8;
+  const int threads = 256;                               // 64 groups per block (four lanes each)
+  int64_t blocks = (groups + 63) / 64;
+  const int64_t cap = static_cast<int64_t>(sm_count) * 16;
   if (blocks > cap) blocks = cap;
   w4::repack_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-      reinterpret_cast<const uint4*>(w), groups, reinterpret_cast<uint4*>(codes), scales, group_m,
-      off_grid_count);
+      reinterpret_cast<const uint4*>(w), groups, codes, scales, group_m, off_grid_count);
   return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
