@@ -155,7 +155,7 @@ __device__ __forceinline__ void compute_sync() {
   asm volatile("bar.sync 1, %0;" ::"r"(kWarps * 32) : "memory");
 }
 
-template <int MT>
+template <int MT, bool GELU>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
                    const __grid_constant__ CUtensorMap tmap_scales, StreamArgs A) {
@@ -280,11 +280,11 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
   // the same j (tile rows 8w+gid and 64+8w+gid), so the gate is applied in registers.  Otherwise
   // 16 consecutive rows per warp.
   const int gid = lane >> 2, tq = lane & 3;
-  const bool gelu = (A.epi == W4_EPI_GELU_GATE);
+  constexpr bool gelu = GELU;
   const int rlo = gelu ? warp * 8 + gid : warp * 16 + gid;
   const int rhi = gelu ? rlo + kHalf : rlo + 8;
   const int r7 = rlo & 7;                       // == rhi & 7
-  const int dw = (rhi - rlo) * 32;              // word distance between the two rows
+  constexpr int kDwBytes = (GELU ? kHalf : 8) * 128;   // byte distance between the two rows
   constexpr int NB = MT / 8;                    // token blocks of 8 (the MMA's n)
   float* ep = reinterpret_cast<float*>(smem + (L.ep_off >= 0 ? L.ep_off : 0));
   int cslot = 0;          // ring slot and mbarrier phase of the current stage
@@ -348,7 +348,10 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       // 128-byte row (TMA 128-byte swizzle).  Each extracted bf16 pair is two consecutive k, so
       // k-step 0 takes elements 8tq+0..3 (x pairs .x, .y) and k-step 1 elements 8tq+4..7 (.z, .w).
       // rows rlo and rhi share the swizzle phase (rlo % 8): one address per group
-      const uint32_t* cwl = cw + rlo * 32 + tq;
+      // shared address of (row rlo, chunk c, word tq) = stage + rlo*128 + ((c ^ r7) << 4) + 4 tq;
+      // the stage and row bases have bits 4-6 clear, so this is base ^ (c << 4) with the r7 part
+      // folded into base: one XOR per group
+      const uint32_t abase = smem_u32(cw) + ((rlo * 128 + 4 * tq) ^ (r7 << 4));
       const bool mask_tail = (A.scale_mode != kScaleTma) && gc < kGS;   // TMA zero-fills past K
 #pragma unroll
       for (int h = 0; h < kGS; h += kGP) {
@@ -357,9 +360,9 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
 #pragma unroll
         for (int i = 0; i < kGP; ++i) {
           const int gi = h + i;
-          const uint32_t* pw = cwl + ((gi ^ r7) << 2);
-          const uint32_t wlo = pw[0];
-          const uint32_t whi = pw[dw];
+          const uint32_t aw = abase ^ static_cast<uint32_t>(gi << 4);
+          const uint32_t wlo = lds32(aw);
+          const uint32_t whi = lds32(aw + kDwBytes);
           // biased codes 128 + u (exact in bf16); the -136 * sum(x) term comes from one MMA per
           // k-step with the constant A = -136, so q * x = (128 + u) * x - 136 * x overall
 #if W4_STREAM_BIASED
@@ -614,22 +617,22 @@ size_t w4_stream_workspace_bytes(int64_t rows, int N, int K, int E, int epi, boo
   return counters_bytes(p, rows) + static_cast<size_t>(p.splits) * rows * N * sizeof(float);
 }
 
-template <int MT>
+template <int MT, bool GELU>
 static w4_status launch_mt(const CUtensorMap& tmap, const CUtensorMap& smap, const w4::StreamArgs& A,
                            int sm_count, cudaStream_t stream) {
   static int attr_done[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(w4::stream_gemm_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(w4::stream_gemm_kernel<MT, GELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              w4::kSmemPerCta) != cudaSuccess)
       return W4_ERR_CUDA;
-    if (cudaFuncSetAttribute(w4::stream_gemm_kernel<MT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+    if (cudaFuncSetAttribute(w4::stream_gemm_kernel<MT, GELU>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return W4_ERR_CUDA;
     attr_done[dev] = 1;
   }
-  w4::stream_gemm_kernel<MT><<<sm_count * w4::kCtasPerSm, w4::kThreads, A.L.total, stream>>>(tmap, smap, A);
+  w4::stream_gemm_kernel<MT, GELU><<<sm_count * w4::kCtasPerSm, w4::kThreads, A.L.total, stream>>>(tmap, smap, A);
   return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
@@ -678,6 +681,10 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
   if (A.scale_mode == w4::kScaleTma &&
       !encode_scales_map(&smap, scales, static_cast<int64_t>(E) * N, A.kg))
     return W4_ERR_CUDA;
-  return p.MT == 8 ? launch_mt<8>(tmap, smap, A, sm_count, stream)
-                   : launch_mt<16>(tmap, smap, A, sm_count, stream);
+  const bool gelu = A.epi == W4_EPI_GELU_GATE;
+  if (p.MT == 8)
+    return gelu ? launch_mt<8, true>(tmap, smap, A, sm_count, stream)
+                : launch_mt<8, false>(tmap, smap, A, sm_count, stream);
+  return gelu ? launch_mt<16, true>(tmap, smap, A, sm_count, stream)
+              : launch_mt<16, false>(tmap, smap, A, sm_count, stream);
 }
