@@ -99,11 +99,16 @@ w4_status w4_repack(const uint16_t* w, int64_t rows, int64_t K, uint32_t* codes,
  *            W4_ERR_WORKSPACE when smaller).  Its contents need no preparation (the call clears
  *            or overwrites the part it relies on, on `stream`).  Calls sharing one workspace must
  *            not overlap on the GPU.
- * y[m, n] = bf16(sum_k x[m, k] * s[n, k/32] * q[n, k]) with float32 accumulation.  Every product
- * x * (s * q) is formed exactly; only the float32 sums and the final rounding are inexact.
+ * y[m, n] = bf16(sum_k x[m, k] * s[n, k/32] * q[n, k]) with float32 accumulation.  Both
+ * kernels first write x once in fp16 with a power-of-two exponent per row (exact for every
+ * element within a factor 2^27 of its row's largest), and every tensor-core product is exact;
+ * the float32 sums and the final rounding are inexact.
  * Two kernels serve the call: for M < 64 (or N % 128 != 0, or K > 4096, or K % 64 != 0) a
- * weight-streaming kernel (workspace: split-K partials), otherwise the tensor-core kernel
- * (workspace: x in fp16 with a power-of-two exponent per row, M * K * 2 bytes plus 4 per row).
+ * weight-streaming kernel (workspace: M * ceil(K/256) * 640 bytes of prepared rows -- fp16
+ * values and per-group bias corrections -- plus 4 per row, and split-K partials), otherwise the
+ * tensor-core kernel (workspace: M * K * 2 bytes plus 4 per row).  In the streaming kernel each
+ * group's sum also carries a float32 rounding of a bias term that its correction cancels: about
+ * 2^-13 of the group's mean |x| times 32 per group, far below the bf16 output rounding.
  */
 w4_status w4a16_linear(const uint16_t* x, const uint32_t* codes, const uint16_t* scales,
                        uint16_t* y, int64_t M, int64_t N, int64_t K, void* workspace,
@@ -145,15 +150,18 @@ w4_status moe_route_permute(const float* logits, int32_t T, int32_t E, int32_t k
  *   rows            total sorted rows (T * k).  N >= 1 (even for W4_EPI_GELU_GATE), K % 32 == 0.
  *   epilogue        W4_EPI_NONE: out [rows, N]; W4_EPI_GELU_GATE: out [rows, N/2].
  *   workspace       at least w4_workspace_bytes(W4_OP_GMM, rows, N, K, E, k) bytes
- *                   (W4_ERR_WORKSPACE when smaller).  Nonzero only when the call takes the
- *                   tensor-core kernel (rows >= 32 * E, K <= 4096, K % 64 == 0, N % 128 == 0 or
- *                   (N/2) % 64 == 0 with W4_EPI_GELU_GATE): every sorted row of `a` in fp16 with
- *                   a power-of-two exponent, rows * K * 2 bytes plus 4 per row.
+ *                   (W4_ERR_WORKSPACE when smaller; nonzero whenever rows > 0): every sorted row
+ *                   of `a` written once, in sorted order, in fp16 with a power-of-two exponent.
+ *                   The tensor-core kernel (rows >= 32 * E, K <= 4096, K % 64 == 0, N % 128 == 0
+ *                   or (N/2) % 64 == 0 with W4_EPI_GELU_GATE) needs rows * K * 2 bytes plus 4
+ *                   per row; the weight-streaming kernel rows * ceil(K/256) * 640 bytes (fp16
+ *                   values and per-group bias corrections) plus 4 per row.
  *   dev_status      one int32 device word or NULL: set to a w4_status code if the device finds a
  *                   problem (offsets out of range: W4_ERR_INVALID_ARG; a pair naming a row past
  *                   the end of `a`: W4_ERR_INVALID_ARG, that row read as row 0); left unchanged
  *                   otherwise.
- * Accumulation is float32 and every product a * (s * q) is exact; out is rounded to bf16.
+ * Accumulation is float32 and every tensor-core product is exact; out is rounded to bf16 (the
+ * accuracy statement of w4a16_linear applies).
  */
 w4_status moe_w4a16_gmm(const uint16_t* a, const int32_t* a_row_of_pair, int32_t k,
                         const uint32_t* codes, const uint16_t* scales,
@@ -175,14 +183,16 @@ w4_status moe_combine(const uint16_t* o, const float* topk_w, const int32_t* pai
  * w4a16_linear_noalloc -- w4a16_linear for callers that cannot allocate device memory.
  * (No counterpart on the pages: an interface addition of this library.)
  *
- * Same arguments, result and accuracy as w4a16_linear, without a workspace: when K is split
- * across CTAs the float32 partials and arrival counters live in a file-scope device array of
- * 8 MiB (8388608 bytes) that every GPU loading the library keeps until process exit.  Callers
+ * Same arguments, result and accuracy as w4a16_linear, without a workspace: the prepared
+ * activation rows and, when K is split across CTAs, the float32 partials and arrival counters
+ * live in a file-scope device array of 8 MiB (8388608 bytes) that every GPU loading the library
+ * keeps until process exit.  Callers
  * that are handed only their input and output buffers (a plugin inside a framework that owns all
  * device memory through its own pool, or a runtime held to a fixed memory budget) can call it
  * without cudaMalloc, which would bypass the pool and synchronise the device.
- *   - Always takes the weight-streaming kernel.  Returns W4_ERR_WORKSPACE when its split-K
- *     scratch for these sizes exceeds 8 MiB (8388608 bytes).
+ *   - Always takes the weight-streaming kernel, over the rows in as many chunks as keep each
+ *     chunk's scratch within 8 MiB.  Returns W4_ERR_WORKSPACE, launching nothing, when a single
+ *     row's scratch exceeds 8 MiB (8388608 bytes).
  *   - The first call on a device looks up the array's device address (once per device); make
  *     that first call before any stream capture.
  *   - Every call reuses the same array (clearing its arrival counters with a cudaMemsetAsync on

@@ -38,11 +38,32 @@ def test_noalloc_matches_workspace_entry_point(M):
         assert_rows_close(host_f64(y), ref)
 
 
-def test_noalloc_rejects_sizes_beyond_its_scratch():
+def test_noalloc_splits_rows_that_do_not_fit_its_scratch():
+    """63 rows against K = 65536: the prepared activation rows alone (640 bytes per 256 k per
+    row) exceed the 8 MiB array, so the call runs the rows in chunks; the result must match the
+    regular entry point."""
     lib = _lib.load()
-    # 64 rows against a 32768 x 16384 weight split K in two: 2 x 64 x 32768 float32 partials are
-    # 16 MiB, over the fixed 8 MiB, so the call must refuse before launching anything
-    M, N, K = 64, 32768, 16384
+    M, N, K = 63, 256, 65536
+    need = api.w4_workspace_bytes(_lib.W4_OP_LINEAR, M, N, K, 1, 1)
+    assert need > api.NOALLOC_SCRATCH_BYTES
+    case = synth.dense_case(M, N, K, 0.01, 1e-4, seed=11)
+    x, codes, scales = dev_bf16(case.x), dev_u32(case.codes), dev_bf16(case.scales)
+    ref = host_f64(api.w4a16_linear(x, codes, scales))
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    st = C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    status = lib.w4a16_linear_noalloc(C.c_void_p(x.data_ptr()), C.c_void_p(codes.data_ptr()),
+                                      C.c_void_p(scales.data_ptr()), C.c_void_p(y.data_ptr()),
+                                      M, N, K, st)
+    assert status == _lib.W4_OK, lib.w4_status_str(status)
+    torch.cuda.synchronize()
+    assert_rows_close(host_f64(y), ref)
+
+
+def test_noalloc_rejects_a_row_beyond_its_scratch():
+    lib = _lib.load()
+    # K = 2^22: one prepared row is 10 MiB, over the fixed 8 MiB, so the call must refuse before
+    # launching anything (the dummy buffers are never touched)
+    M, N, K = 1, 8, 1 << 22
     need = api.w4_workspace_bytes(_lib.W4_OP_LINEAR, M, N, K, 1, 1)
     assert need > api.NOALLOC_SCRATCH_BYTES
     dummy = torch.empty(16, dtype=torch.uint8, device="cuda")

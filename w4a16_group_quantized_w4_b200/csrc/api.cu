@@ -96,12 +96,18 @@ size_t w4_workspace_bytes(int32_t op, int64_t M_or_T, int64_t N, int64_t K, int3
     case W4_OP_ROUTE:
       return w4_route_workspace_bytes(static_cast<int>(M_or_T), E);
     case W4_OP_GMM: {
-      // the tensor-core path writes every routed row in fp16, in pair order; the streaming path
-      // needs nothing
+      // both paths write every routed row once, in pair order, in their own prepared form; the
+      // size covers whichever path either epilogue takes
       if (N <= 0 || K < 32 || K % 32 || E < 1 || N > (1LL << 30) || K > (1LL << 30)) return 0;
-      const bool tc = use_tc(M_or_T, E, static_cast<int>(N), static_cast<int>(K), W4_EPI_NONE, false, nullptr) ||
-                      use_tc(M_or_T, E, static_cast<int>(N), static_cast<int>(K), W4_EPI_GELU_GATE, false, nullptr);
-      return tc ? w4_tc_workspace_bytes(M_or_T, static_cast<int>(K)) : 0;
+      size_t need = 0;
+      for (int epi : {W4_EPI_NONE, W4_EPI_GELU_GATE}) {
+        const size_t b = use_tc(M_or_T, E, static_cast<int>(N), static_cast<int>(K), epi, false, nullptr)
+                             ? w4_tc_workspace_bytes(M_or_T, static_cast<int>(K))
+                             : w4_stream_workspace_bytes(M_or_T, static_cast<int>(N), static_cast<int>(K), E,
+                                                         epi, false, current_sm_count());
+        if (b > need) need = b;
+      }
+      return need;
     }
     default:
       return 0;

@@ -137,39 +137,43 @@ __device__ __forceinline__ uint16_t ldg_u16(const uint16_t* p) {
 }
 
 // ------------------------------------------------------------------------------------------
-// int4 -> bf16 dequantisation of nibble pairs, and the warp-level bf16 MMA
+// power-of-two row exponents, int4 -> fp16 nibble extraction and the warp-level fp16 MMA
 // ------------------------------------------------------------------------------------------
 
-// Takes bits 0..3 and 16..19 of v (two 4-bit fields u), returns the bf16 pair (u - 8).
-// 0x4300 | u is the bf16 value 128 + u; one packed fma subtracts 136 exactly.
-__device__ __forceinline__ uint32_t nibbles_to_bf16x2(uint32_t v) {
-  uint32_t r, q;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(v), "r"(0x000F000Fu), "r"(0x43004300u));
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(q) : "r"(r), "r"(0x3F803F80u), "r"(0xC308C308u));
-  return q;
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }   // |e| <= 126
+
+// Power-of-two exponent that brings a finite magnitude with bf16 bit pattern m (sign cleared) to
+// [2^(top), 2^(top+1)); 0 for m == 0.  Clamped to +-100 so that 2^e and 2^-e stay normal floats.
+__device__ __forceinline__ int shift_for(uint32_t m, int top) {
+  if (m == 0) return 0;
+  int E = static_cast<int>(m >> 7);
+  if (E == 0) E = 1;                                   // subnormal: below 2^-126
+  int e = top + 127 - E;
+  return e < -100 ? -100 : (e > 100 ? 100 : e);
 }
 
-// Same fields, returned biased: the bf16 pair (128 + u), exact.  A caller that multiplies these
-// by x must subtract 136 * sum(x) (see kMinus136x2).
-__device__ __forceinline__ uint32_t nibbles_to_bf16x2_biased(uint32_t v) {
+
+// Nibble fields of a layout-L1 code word as exact fp16 pairs, without a subtraction: OR-ing a
+// field into the mantissa of 1024 (0x6400, unit in the last place 1) gives 1024 + u when the field
+// sits at bits 0..3 of each half, 1024 + 16 u at bits 4..7.  The bias (1024, or 1024 / 16 once the
+// matching activation is pre-divided by 16) and the -8 of q = u - 8 are removed by a per-group
+// correction that enters the MMA as its C operand.
+__device__ __forceinline__ uint32_t nib_f16x2_lo(uint32_t v) {   // bits 0..3 | 16..19 -> 1024 + u
   uint32_t r;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(v), "r"(0x000F000Fu), "r"(0x43004300u));
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(v), "r"(0x000F000Fu), "r"(0x64006400u));
+  return r;
+}
+__device__ __forceinline__ uint32_t nib_f16x2_hi(uint32_t v) {   // bits 4..7 | 20..23 -> 1024 + 16u
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(v), "r"(0x00F000F0u), "r"(0x64006400u));
   return r;
 }
 
-constexpr uint32_t kMinus136x2 = 0xC308C308u;   // bf16 pair (-136, -136)
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t r;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
-  return r;
-}
-
-// D = A(16x16 bf16, row) * B(16x8 bf16, col) + C, float32 accumulators.
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
-                                               uint32_t b0, uint32_t b1, const float (&c)[4]) {
+// D = A(16x16 fp16, row) * B(16x8 fp16, col) + C, float32 accumulators.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1, const float (&c)[4]) {
   asm(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
       "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %11, %12, %13};"
       : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1),

@@ -4,8 +4,9 @@
 // custom-op hook inside a host framework that owns every device byte through its own pool (a
 // cudaMalloc there escapes the pool's accounting and synchronises the whole device, stalling
 // other work), or a runtime that must run inside a fixed, pre-reserved memory budget.  The
-// regular w4a16_linear asks them for a workspace when it splits K across CTAs; this entry point
-// takes that scratch from a file-scope device array instead, so nothing is allocated per call.
+// regular w4a16_linear asks them for a workspace (prepared activation rows, split-K partials);
+// this entry point takes that scratch from a file-scope device array instead, so nothing is
+// allocated per call, and runs the rows in as many chunks as the array needs.
 //
 // The array is kNoallocScratchBytes (8 MiB) and every GPU that loads the library keeps it until
 // the process exits.  Its address is looked up once per device with cudaGetSymbolAddress (the
@@ -23,8 +24,8 @@ namespace {
 
 constexpr size_t kNoallocScratchBytes = size_t(8) << 20;
 
-// Split-K arrival counters followed by the float32 partials.  Zero at module load; the counters
-// are cleared again by every call that splits K.
+// Prepared activation rows, then split-K arrival counters and float32 partials.  Zero at module
+// load; the counters are cleared again by every call that splits K.
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -74,19 +75,28 @@ w4_status w4a16_linear_noalloc(const uint16_t* x, const uint32_t* codes, const u
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return W4_ERR_CUDA;
-  const size_t need = w4_stream_workspace_bytes(M, static_cast<int>(N), static_cast<int>(K), 1,
-                                                W4_EPI_NONE, true, sms);
-  if (need > kNoallocScratchBytes) return W4_ERR_WORKSPACE;   // larger than the fixed scratch
+  // rows in chunks whose workspace (prepared activation rows, split-K partials) fits the scratch
+  auto need_for = [&](int64_t rows) {
+    return w4_stream_workspace_bytes(rows, static_cast<int>(N), static_cast<int>(K), 1, W4_EPI_NONE,
+                                     true, sms);
+  };
+  if (M == 0) return W4_OK;
+  int64_t chunk = M;
+  while (chunk > 1 && need_for(chunk) > kNoallocScratchBytes) chunk = (chunk + 1) / 2;
+  if (need_for(chunk) > kNoallocScratchBytes) return W4_ERR_WORKSPACE;   // one row is too large
+  cudaError_t err;
+  void* ws = scratch_for_current_device(&err);
+  if (!ws) return W4_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  void* ws = nullptr;
-  if (need > 0) {
-    cudaError_t err;
-    ws = scratch_for_current_device(&err);
-    if (!ws) return W4_ERR_CUDA;
-    // (the launch clears the split-K arrival counters at the head of the scratch itself)
+  for (int64_t r0 = 0; r0 < M; r0 += chunk) {
+    const int64_t rows = M - r0 < chunk ? M - r0 : chunk;
+    // (each launch clears the split-K arrival counters it uses)
+    const w4_status st = w4_launch_stream_gemm(x + r0 * K, nullptr, 1, codes, scales, nullptr, 1, rows,
+                                               static_cast<int>(N), static_cast<int>(K), W4_EPI_NONE,
+                                               y + r0 * N, ws, kNoallocScratchBytes, nullptr, s, sms);
+    if (st != W4_OK) return st;
   }
-  return w4_launch_stream_gemm(x, nullptr, 1, codes, scales, nullptr, 1, M, static_cast<int>(N),
-                               static_cast<int>(K), W4_EPI_NONE, y, ws, need, nullptr, s, sms);
+  return W4_OK;
 }
 
 }  // extern "C"

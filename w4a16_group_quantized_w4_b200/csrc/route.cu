@@ -15,7 +15,8 @@
 //            and each warp walks a contiguous run of pairs: a per-warp histogram pass, a scan of
 //            the warp bases, then positions from __match_any_sync ranks.  Positions are exact and
 //            independent of scheduling.
-//   Small T runs both phases in one CTA (one launch); large T uses two launches.
+//   Small T (<= 128) runs in one CTA (one launch) with per-expert token bit masks instead of the
+//   scatter (route_fused_kernel); large T uses two launches.
 #include "common.cuh"
 
 namespace w4 {
@@ -38,56 +39,67 @@ struct RouteArgs {
   int scatter_warps;    // warps taking part in the scatter (shared scratch scales with it)
 };
 
-__device__ __forceinline__ bool better(float v, int i, float w, int j) {
-  return v > w || (v == w && i < j);
+// Order-preserving map of a non-NaN float to uint32 (larger value -> larger key); -0 and +0 map
+// to the same key, so equal logits compare equal exactly as they do as floats.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t b = __float_as_uint(v + 0.0f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// Top-k for tokens [t0, t1) of this CTA; accumulates counts into s_cnt[E] (shared).
-// PL = logits per lane (E <= 32 * PL); lane l holds experts c * 32 + l.
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// Top-k of token t by one warp; writes topk_ids / topk_w and returns, in lanes 0..k-1, the
+// expert chosen in round `lane` (-1 in the other lanes).
+// PL = logits per lane (E <= 32 * PL); lane l holds experts c * 32 + l as order keys.  Each round
+// takes the warp maximum of the lanes' best untaken keys (one redux), then the lowest expert
+// index among the lanes holding it (a second redux).
+template <int PL>
+__device__ int topk_token(const RouteArgs& A, int t) {
+  const int lane = threadIdx.x & 31;
+  uint32_t key[PL];
+  const float* row = A.logits + static_cast<int64_t>(t) * A.E;
+#pragma unroll
+  for (int c = 0; c < PL; ++c) {
+    const int e = c * 32 + lane;
+    key[c] = e < A.E ? order_key(__ldg(row + e)) : 0u;     // 0: below every real key
+  }
+  uint32_t taken = 0;
+  uint32_t top = 0, sel_key = 0;
+  int sel_e = -1;
+  for (int j = 0; j < A.k; ++j) {
+    uint32_t bk = 0;
+    int be = 0x7FFFFFFF;
+#pragma unroll
+    for (int c = 0; c < PL; ++c) {                    // ascending c: the first maximum is the
+      const bool free_c = !((taken >> c) & 1u);         // lowest index of this lane
+      if (free_c && key[c] > bk) { bk = key[c]; be = c * 32 + lane; }
+    }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    const int win = static_cast<int>(__reduce_min_sync(0xffffffffu, bk == m ? static_cast<uint32_t>(be)
+                                                                          : 0x7FFFFFFFu));
+    if ((win & 31) == lane) taken |= 1u << (win >> 5);
+    if (j == 0) top = m;
+    if (lane == j) { sel_key = m; sel_e = win; }
+  }
+  const float ex = lane < A.k ? expf(key_value(sel_key) - key_value(top)) : 0.f;
+  float sum = ex;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane < A.k) {
+    A.topk_ids[static_cast<int64_t>(t) * A.k + lane] = sel_e;
+    A.topk_w[static_cast<int64_t>(t) * A.k + lane] = ex / sum;
+  }
+  return sel_e;
+}
+
 template <int PL>
 __device__ void topk_tokens(const RouteArgs& A, int t0, int t1, int* s_cnt) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   for (int t = t0 + warp; t < t1; t += nwarps) {
-    float v[PL];
-    const float* row = A.logits + static_cast<int64_t>(t) * A.E;
-#pragma unroll
-    for (int c = 0; c < PL; ++c) {
-      const int e = c * 32 + lane;
-      v[c] = e < A.E ? __ldg(row + e) : -INFINITY;
-    }
-    uint32_t taken = 0;
-    float sel_v = 0.f, top = 0.f;
-    int sel_e = 0;
-    for (int j = 0; j < A.k; ++j) {
-      float bv = -INFINITY;
-      int be = 0x7FFFFFFF;
-#pragma unroll
-      for (int c = 0; c < PL; ++c) {
-        const int e = c * 32 + lane;
-        if (e < A.E && !((taken >> c) & 1u) && better(v[c], e, bv, be)) {
-          bv = v[c];
-          be = e;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (better(ov, oe, bv, be)) { bv = ov; be = oe; }
-      }
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      if (j == 0) top = bv;
-      if (lane == j) { sel_v = bv; sel_e = be; }
-    }
-    const float ex = lane < A.k ? expf(sel_v - top) : 0.f;
-    float sum = ex;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane < A.k) {
-      A.topk_ids[static_cast<int64_t>(t) * A.k + lane] = sel_e;
-      A.topk_w[static_cast<int64_t>(t) * A.k + lane] = ex / sum;
-      atomicAdd(&s_cnt[sel_e], 1);
-    }
+    const int e = topk_token<PL>(A, t);
+    if (lane < A.k) atomicAdd(&s_cnt[e], 1);
   }
 }
 
@@ -155,27 +167,83 @@ __device__ __forceinline__ void topk_dispatch(const RouteArgs& A, int t0, int t1
   else topk_tokens<32>(A, t0, t1, s_cnt);
 }
 
-// One CTA does everything (small T).
+template <int PL>
+__device__ void fused_topk(const RouteArgs& A, int* s_ids, uint32_t* s_mask, int W) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int t = warp; t < A.T; t += nwarps) {
+    const int e = topk_token<PL>(A, t);
+    if (lane < A.k) {
+      s_ids[t * A.k + lane] = e;
+      atomicOr(&s_mask[e * W + (t >> 5)], 1u << (t & 31));
+    }
+  }
+}
+
+// One CTA does everything (T <= kFusedMaxT).  A token picks an expert at most once, so the
+// tokens routed to expert e form a T-bit mask, and the rank of pair (t, j) among expert e's
+// pairs -- ordered by pair id, i.e. by token -- is the number of mask bits below t:
+//   offsets     exclusive scan over e of popcount(mask[e])      (one thread per expert)
+//   positions   pos(t, j) = offsets[e] + popcount(mask[e] & bits below t)   (one thread per pair)
+// Every step is a parallel pass; no serial loop over experts or warps.
 __global__ void __launch_bounds__(kFusedWarps * 32) route_fused_kernel(RouteArgs A) {
   extern __shared__ int smem[];
-  int* s_cnt = smem;                     // [E]
-  int* s_base = s_cnt + A.E;             // [E]
-  int* s_wcnt = s_base + A.E;            // [nwarps][E]
-  for (int e = threadIdx.x; e < A.E; e += blockDim.x) s_cnt[e] = 0;
+  const int W = (A.T + 31) >> 5;                          // mask words per expert (<= 4)
+  uint32_t* s_mask = reinterpret_cast<uint32_t*>(smem);   // [E][W]
+  int* s_off = smem + A.E * W;                            // [E]
+  int* s_ids = s_off + A.E;                               // [T][k]
+  int* s_wsum = s_ids + A.T * A.k;                        // [32]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < A.E * W; i += blockDim.x) s_mask[i] = 0u;
   __syncthreads();
-  topk_dispatch(A, 0, A.T, s_cnt);
+  if (A.E <= 32) fused_topk<1>(A, s_ids, s_mask, W);
+  else if (A.E <= 64) fused_topk<2>(A, s_ids, s_mask, W);
+  else if (A.E <= 128) fused_topk<4>(A, s_ids, s_mask, W);
+  else if (A.E <= 256) fused_topk<8>(A, s_ids, s_mask, W);
+  else if (A.E <= 512) fused_topk<16>(A, s_ids, s_mask, W);
+  else fused_topk<32>(A, s_ids, s_mask, W);
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int e = 0; e < A.E; ++e) {
-      s_base[e] = run;
-      A.expert_offsets[e] = run;
-      run += s_cnt[e];
+  // exclusive scan of the per-expert counts (E <= blockDim.x)
+  const int e = threadIdx.x;
+  int cnt = 0;
+  if (e < A.E)
+    for (int w = 0; w < W; ++w) cnt += __popc(s_mask[e * W + w]);
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) s_wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int v = s_wsum[lane];
+    int wi = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += u;
     }
-    A.expert_offsets[A.E] = run;
+    s_wsum[lane] = wi - v;                                // exclusive over warps
   }
   __syncthreads();
-  scatter_pairs(A, 0, static_cast<int64_t>(A.T) * A.k, s_base, s_wcnt, A.scatter_warps);
+  if (e < A.E) {
+    const int off = s_wsum[warp] + incl - cnt;
+    s_off[e] = off;
+    A.expert_offsets[e] = off;
+    if (e == A.E - 1) A.expert_offsets[A.E] = off + cnt;
+  }
+  __syncthreads();
+  const int P = A.T * A.k;
+  for (int p = threadIdx.x; p < P; p += blockDim.x) {
+    const int t = p / A.k;
+    const int ex = s_ids[p];
+    const uint32_t* m = s_mask + ex * W;
+    int rank = __popc(m[t >> 5] & ((1u << (t & 31)) - 1u));
+    for (int w = 0; w < (t >> 5); ++w) rank += __popc(m[w]);
+    const int pos = s_off[ex] + rank;
+    A.sorted_pair[pos] = p;
+    A.pair_pos[p] = pos;
+  }
 }
 
 __global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(RouteArgs A) {
@@ -314,8 +382,9 @@ w4_status w4_launch_route(const float* logits, int T, int E, int k, int32_t* ids
     return W4_OK;
   }
   if (w4_route_workspace_bytes(T, E) == 0) {
-    A.scatter_warps = scatter_warps_for(E, w4::kFusedWarps);
-    const size_t smem = static_cast<size_t>(2 + A.scatter_warps) * E * sizeof(int);
+    // masks [E][ceil(T/32)], offsets [E], ids [T][k], warp sums [32]: <= 36 KB (E <= 1024)
+    const size_t smem = (static_cast<size_t>(E) * ((T + 31) / 32) + E + static_cast<size_t>(T) * k + 32) *
+                        sizeof(int);
     w4::route_fused_kernel<<<1, w4::kFusedWarps * 32, smem, stream>>>(A);
   } else {
     if (ws == nullptr || ws_bytes < w4_route_workspace_bytes(T, E)) return W4_ERR_WORKSPACE;

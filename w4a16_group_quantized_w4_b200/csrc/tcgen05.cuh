@@ -113,18 +113,6 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }   // |e| <= 126
-
-// Power-of-two exponent that brings a finite magnitude with bf16 bit pattern m (sign cleared) to
-// [2^(top), 2^(top+1)); 0 for m == 0.  Clamped to +-100 so that 2^e and 2^-e stay normal floats.
-__device__ __forceinline__ int shift_for(uint32_t m, int top) {
-  if (m == 0) return 0;
-  int E = static_cast<int>(m >> 7);
-  if (E == 0) E = 1;                                   // subnormal: below 2^-126
-  int e = top + 127 - E;
-  return e < -100 ? -100 : (e > 100 ? 100 : e);
-}
-
 }  // namespace w4
 
 // Conversion pass in front of the tensor-core kernels (convert.cu): row p of a16 becomes the
