@@ -39,7 +39,7 @@ def test_noalloc_matches_workspace_entry_point(M):
 
 
 def test_noalloc_splits_rows_that_do_not_fit_its_scratch():
-    """63 rows against K = 65536: the prepared activation rows alone (640 bytes per 256 k per
+    """63 rows against K = 65536: the prepared activation rows alone (656 bytes per 256 k per
     row) exceed the 8 MiB array, so the call runs the rows in chunks; the result must match the
     regular entry point."""
     lib = _lib.load()

@@ -11,9 +11,10 @@
 // Design (sm_100a):
 //   * A preparation pass (one warp per routed row) writes each activation row once, gathered into
 //     routed-row order, as fp16 with a power-of-two exponent per row: x' = x * 2^f, f putting the
-//     row's largest |x| in [2^14, 2^15), and rowmul = 2^-f.  Within every 8 consecutive k the
-//     elements 2, 3, 6, 7 are stored divided by 16 (see the dequantisation below).  Next to each
-//     256-k block of a row it stores the block's 8 group corrections
+//     row's largest |x| in [2^14, 2^15), with the multiplier 2^-f beside every 256-k block.
+//     Within every 8 consecutive k the elements 2, 3, 6, 7 are stored divided by 16 (see the
+//     dequantisation below).  Next to each 256-k block of a row it stores the block's 8 group
+//     corrections
 //     c = -(1032 * sum of x' over elements 0, 1, 4, 5 + 1152 * sum of the stored x'/16 values),
 //     as quads {c(r), c(r + 1), c(r), c(r + 1)} for the row pair (r, r + 1).
 //   * Work unit = (expert e, block of <= MT routed rows (MT = 8 or 16), tile of 128 weight rows,
@@ -33,7 +34,8 @@
 //     bias and the -8 of q = u - 8: d = sum over the group of q * x'.  The packed nibble order
 //     puts two consecutive k in each extracted pair, so the activation B fragments are plain
 //     16-byte shared loads.  The group's scale is folded in with one fp32 FMA per accumulator:
-//     acc += s_g * d.  The epilogue multiplies by the token's rowmul.
+//     acc += s_g * d.  The epilogue multiplies by the token's 2^-f, read from the unit's last
+//     stage (a global load there would wait behind the weight stream).
 //   * Epilogue from registers, without a CTA barrier: with the GELU gate each warp's two A-fragment
 //     row sets are 8 gate rows and the 8 up rows of the same outputs, so h = gelu(g) * u is formed
 //     in the thread that holds both.  Dense split-K writes float32 partials that the last CTA of
@@ -67,8 +69,9 @@ constexpr int kBN = 16 * kWarps;              // weight rows per tile
 constexpr int kHalf = kBN / 2;                // rows per TMA box
 constexpr int kXPitch = kGS * 64 + 64;        // bytes per token row in an activation stage
 constexpr int kXBlock = kGS * 64;             // prepared activation bytes per row and stage
+constexpr int kXCopy = kXBlock + 16;          // + the row's multiplier 2^-f (and 12 spare bytes)
 constexpr int kQBlock = kGS * 16;             // correction-quad bytes per row and stage
-constexpr int kPrepStage = kXBlock + kQBlock; // prepared bytes per row and 256-k block (640)
+constexpr int kPrepStage = kXCopy + kQBlock;  // prepared bytes per row and 256-k block (656)
 constexpr int kQPitch = kQBlock + 16;         // bytes per row pair in a stage's quad area
 constexpr int kCodeBytes = kBN * kGS * 16;    // 16 KB
 constexpr int kBlockMaxKg = 24;               // scale-block mode: two 64-row blocks of <= 24 groups
@@ -96,9 +99,8 @@ struct Layout {
 };
 
 struct StreamArgs {
-  const uint8_t* xw;        // prepared rows: [rows][kstages][640 bytes] (fp16 x', quads)
+  const uint8_t* xw;        // prepared rows: [rows][kstages][656 bytes] (fp16 x', 2^-f, quads)
   int64_t xw_stride;        // bytes per prepared row
-  const float* rowmul;      // [rows] 2^-f
   const uint16_t* scales;   // [E*N, kg]
   const int32_t* offsets;   // [E+1] or null (one expert with `rows` rows)
   int E, N, K, kg;
@@ -311,7 +313,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           else if (SCALE == kScaleBlock) sbytes = 2 * kHalf * A.kg * 2;
           // whole 256-k blocks of every row (the preparation pass zero-fills past K) and the
           // quads of the even rows; the arrive releases the descriptor written above
-          mbar_arrive_expect_tx(&full[slot], kCodeBytes + sbytes + kXBlock * U.mt + kQBlock * ((U.mt + 1) >> 1));
+          mbar_arrive_expect_tx(&full[slot], kCodeBytes + sbytes + kXCopy * U.mt + kQBlock * ((U.mt + 1) >> 1));
           tma_load_2d(cdst, &tmap_codes, g * 4, static_cast<int32_t>(row_a), &full[slot]);
           tma_load_2d(cdst + kHalf * 128, &tmap_codes, g * 4, static_cast<int32_t>(row_b), &full[slot]);
           if (SCALE == kScaleTma) {
@@ -326,8 +328,8 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         __syncwarp();
         if (lane < U.mt) {
           const uint8_t* blk = xsrc + static_cast<int64_t>(g / kGS) * kPrepStage;
-          bulk_g2s(xdst + lane * kXPitch, blk, kXBlock, &full[slot]);
-          if (!(lane & 1)) bulk_g2s(qdst + (lane >> 1) * kQPitch, blk + kXBlock, kQBlock, &full[slot]);
+          bulk_g2s(xdst + lane * kXPitch, blk, kXCopy, &full[slot]);
+          if (!(lane & 1)) bulk_g2s(qdst + (lane >> 1) * kQPitch, blk + kXCopy, kQBlock, &full[slot]);
         }
         advance();
       }
@@ -502,22 +504,26 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         }
       }
     }
+    const bool last = dsc.flags & kDescLast;
+    if (last) {
+      // undo the activation rows' power-of-two exponents (token columns 2tq, 2tq + 1 of each
+      // block; the multipliers travel with the rows, so no global load waits behind the stream)
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const int t0 = b * 8 + 2 * tq;
+        const float m0 = t0 < mt ? *reinterpret_cast<const float*>(xs + t0 * kXPitch + kXBlock) : 0.f;
+        const float m1 = t0 + 1 < mt ? *reinterpret_cast<const float*>(xs + (t0 + 1) * kXPitch + kXBlock) : 0.f;
+        acc[b][0] *= m0; acc[b][2] *= m0;
+        acc[b][1] *= m1; acc[b][3] *= m1;
+      }
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
-    if (!(dsc.flags & kDescLast)) continue;
+    if (!last) continue;
 
     // --------------------------- epilogue (last stage of a unit) ---------------------------
     const int64_t r0 = dsc.r0;
     const int nt = dsc.nt;
-    // undo the activation rows' power-of-two exponents (token columns 2tq, 2tq + 1 of each block)
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      const int t0 = b * 8 + 2 * tq;
-      const float m0 = t0 < mt ? __ldg(A.rowmul + r0 + t0) : 0.f;
-      const float m1 = t0 + 1 < mt ? __ldg(A.rowmul + r0 + t0 + 1) : 0.f;
-      acc[b][0] *= m0; acc[b][2] *= m0;
-      acc[b][1] *= m1; acc[b][3] *= m1;
-    }
     if (A.splits == 1) {
       // straight from registers: thread holds rows rlo / rhi for tokens 2tq, 2tq + 1 of each block
 #pragma unroll
@@ -605,11 +611,12 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
 // (elements 2, 3, 6, 7 with 2^(f-4), the rest with 2^f) and the correction of group l / 4:
 // c = -(1032 * (x'0 + x'1 + x'4 + x'5) + 1152 * (x'2 + x'3 + x'6 + x'7)) summed over its 4 lanes
 // (from the stored fp16 values), into the quad slots 0, 2 of row r and 1, 3 of row r - 1.
-// Elements past K are written as zero.  rowmul[r] = 2^-f.
+// Elements past K are written as zero.  Every block also carries the row's multiplier 2^-f
+// (bytes 512..515), so that a unit's epilogue finds it next to its last stage.
 __global__ void __launch_bounds__(256)
 stream_prep_kernel(const uint16_t* __restrict__ a, const int32_t* __restrict__ a_row_of_pair, int k_div,
                    int64_t a_rows, int64_t rows, int K, uint8_t* __restrict__ xw, int64_t stride,
-                   float* __restrict__ rowmul, int32_t* dev_status) {
+                   int32_t* dev_status) {
   const int lane = threadIdx.x & 31;
   const int64_t wpb = blockDim.x >> 5;
   const int nv = K >> 3;                          // 8-element chunks in the row
@@ -661,18 +668,20 @@ stream_prep_kernel(const uint16_t* __restrict__ a, const int32_t* __restrict__ a
       part += __shfl_xor_sync(0xffffffffu, part, 2);
       if ((lane & 3) == 0) {
         const float c = -part;
-        float* q = reinterpret_cast<float*>(blk + kXBlock + (lane >> 2) * 16);
+        float* q = reinterpret_cast<float*>(blk + kXCopy + (lane >> 2) * 16);
         q[0] = c;
         q[2] = c;
         if (r + 1 == rows) { q[1] = 0.f; q[3] = 0.f; }
         if (r > 0) {
-          float* qp = reinterpret_cast<float*>(blk - stride + kXBlock + (lane >> 2) * 16);
+          float* qp = reinterpret_cast<float*>(blk - stride + kXCopy + (lane >> 2) * 16);
           qp[1] = c;
           qp[3] = c;
         }
       }
     }
-    if (lane == 0) rowmul[r] = pow2f(-f);
+    for (int j = lane; j < nblk; j += 32)
+      *reinterpret_cast<float4*>(dst + static_cast<int64_t>(j) * kPrepStage + kXBlock) =
+          make_float4(pow2f(-f), 0.f, 0.f, 0.f);
   }
 }
 
@@ -787,9 +796,9 @@ static StreamPlan plan_stream(int64_t rows, int N, int K, int E, int epi, bool d
   return p;
 }
 
-// Workspace: the prepared activation rows [rows][K/256 blocks][640 bytes] and rowmul [rows]
-// (each 256-byte aligned); with split-K then the per-tile arrival counters (cleared by every
-// launch) and the float32 partials [splits, rows, N].
+// Workspace: the prepared activation rows [rows][K/256 blocks][656 bytes] (256-byte aligned);
+// with split-K then the per-tile arrival counters (cleared by every launch) and the float32
+// partials [splits, rows, N].
 static size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
 static int64_t prep_stride(int K) {
@@ -797,7 +806,7 @@ static int64_t prep_stride(int K) {
 }
 
 static size_t prep_bytes(int64_t rows, int K) {
-  return align256(static_cast<size_t>(rows) * prep_stride(K)) + align256(static_cast<size_t>(rows) * 4);
+  return align256(static_cast<size_t>(rows) * prep_stride(K));
 }
 
 static size_t counters_bytes(const StreamPlan& p, int64_t rows) {
@@ -871,7 +880,6 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   A.xw = wsb;
   A.xw_stride = prep_stride(K);
-  A.rowmul = reinterpret_cast<const float*>(wsb + align256(static_cast<size_t>(rows) * A.xw_stride));
   if (p.splits > 1) {
     uint8_t* cbase = wsb + prep_bytes(rows, K);
     const size_t cb = counters_bytes(p, rows);
@@ -886,8 +894,7 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
     const int64_t blocks = (rows + 7) / 8;
     const int grid = static_cast<int>(blocks < 16LL * sm_count ? blocks : 16LL * sm_count);
     w4::stream_prep_kernel<<<grid, 256, 0, stream>>>(a, a_row_of_pair, kd, a_rows, rows, K, wsb,
-                                                     A.xw_stride, const_cast<float*>(A.rowmul),
-                                                     dev_status);
+                                                     A.xw_stride, dev_status);
     if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
   }
   CUtensorMap tmap, smap;
