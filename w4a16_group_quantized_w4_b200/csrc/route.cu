@@ -50,19 +50,18 @@ __device__ __forceinline__ float key_value(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
 }
 
-// Top-k of token t by one warp; writes topk_ids / topk_w and returns, in lanes 0..k-1, the
-// expert chosen in round `lane` (-1 in the other lanes).
-// PL = logits per lane (E <= 32 * PL); lane l holds experts c * 32 + l as order keys.  Each round
-// takes the warp maximum of the lanes' best untaken keys (one redux), then the lowest expert
-// index among the lanes holding it (a second redux).
-template <int PL>
-__device__ int topk_token(const RouteArgs& A, int t) {
-  const int lane = threadIdx.x & 31;
+// Top-k of token t by a group of G lanes (a warp, or a half warp with mask gmask); writes
+// topk_ids / topk_w and returns, in group lanes 0..k-1, the expert chosen in round `gl` (-1 in
+// the other lanes).  PL = logits per lane (E <= G * PL); group lane gl holds experts c * G + gl
+// as order keys.  Each round takes the group maximum of the lanes' best untaken keys (one
+// redux), then the lowest expert index among the lanes holding it (a second redux).
+template <int PL, int G>
+__device__ int topk_token(const RouteArgs& A, int t, uint32_t gmask, int gl) {
   uint32_t key[PL];
   const float* row = A.logits + static_cast<int64_t>(t) * A.E;
 #pragma unroll
   for (int c = 0; c < PL; ++c) {
-    const int e = c * 32 + lane;
+    const int e = c * G + gl;
     key[c] = e < A.E ? order_key(__ldg(row + e)) : 0u;     // 0: below every real key
   }
   uint32_t taken = 0;
@@ -74,32 +73,57 @@ __device__ int topk_token(const RouteArgs& A, int t) {
 #pragma unroll
     for (int c = 0; c < PL; ++c) {                    // ascending c: the first maximum is the
       const bool free_c = !((taken >> c) & 1u);         // lowest index of this lane
-      if (free_c && key[c] > bk) { bk = key[c]; be = c * 32 + lane; }
+      if (free_c && key[c] > bk) { bk = key[c]; be = c * G + gl; }
     }
-    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
-    const int win = static_cast<int>(__reduce_min_sync(0xffffffffu, bk == m ? static_cast<uint32_t>(be)
-                                                                          : 0x7FFFFFFFu));
-    if ((win & 31) == lane) taken |= 1u << (win >> 5);
+    const uint32_t m = __reduce_max_sync(gmask, bk);
+    const int win = static_cast<int>(__reduce_min_sync(gmask, bk == m ? static_cast<uint32_t>(be) : 0x7FFFFFFFu));
+    if ((win % G) == gl) taken |= 1u << (win / G);
     if (j == 0) top = m;
-    if (lane == j) { sel_key = m; sel_e = win; }
+    if (gl == j) { sel_key = m; sel_e = win; }
   }
-  const float ex = lane < A.k ? expf(key_value(sel_key) - key_value(top)) : 0.f;
+  const float ex = gl < A.k ? expf(key_value(sel_key) - key_value(top)) : 0.f;
   float sum = ex;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane < A.k) {
-    A.topk_ids[static_cast<int64_t>(t) * A.k + lane] = sel_e;
-    A.topk_w[static_cast<int64_t>(t) * A.k + lane] = ex / sum;
+  for (int o = G / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(gmask, sum, o);
+  if (gl < A.k) {
+    A.topk_ids[static_cast<int64_t>(t) * A.k + gl] = sel_e;
+    A.topk_w[static_cast<int64_t>(t) * A.k + gl] = ex / sum;
   }
   return sel_e;
 }
 
-template <int PL>
-__device__ void topk_tokens(const RouteArgs& A, int t0, int t1, int* s_cnt) {
+// Calls f(t, e, gl) for every token t of [t0, t1) after its top-k, with e the expert the group
+// lane gl picked (gl < k).  Half warps (two tokens per warp at once) when k <= 16 and E <= 256.
+template <int PL, int G, typename F>
+__device__ void topk_range(const RouteArgs& A, int t0, int t1, F&& f) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  for (int t = t0 + warp; t < t1; t += nwarps) {
-    const int e = topk_token<PL>(A, t);
-    if (lane < A.k) atomicAdd(&s_cnt[e], 1);
+  constexpr int kPerWarp = 32 / G;
+  const int sub = lane / G, gl = lane % G;
+  const uint32_t gmask = G == 32 ? 0xffffffffu : (0xFFFFu << (16 * sub));
+  for (int base = t0 + warp * kPerWarp; base < t1; base += nwarps * kPerWarp) {
+    const int t = base + sub;
+    if (t < t1) {
+      const int e = topk_token<PL, G>(A, t, gmask, gl);
+      if (gl < A.k) f(t, e, gl);
+    }
+  }
+}
+
+template <typename F>
+__device__ void topk_dispatch(const RouteArgs& A, int t0, int t1, F&& f) {
+  if (A.k <= 16 && A.E <= 256) {
+    if (A.E <= 16) topk_range<1, 16>(A, t0, t1, f);
+    else if (A.E <= 32) topk_range<2, 16>(A, t0, t1, f);
+    else if (A.E <= 64) topk_range<4, 16>(A, t0, t1, f);
+    else if (A.E <= 128) topk_range<8, 16>(A, t0, t1, f);
+    else topk_range<16, 16>(A, t0, t1, f);
+  } else {
+    if (A.E <= 32) topk_range<1, 32>(A, t0, t1, f);
+    else if (A.E <= 64) topk_range<2, 32>(A, t0, t1, f);
+    else if (A.E <= 128) topk_range<4, 32>(A, t0, t1, f);
+    else if (A.E <= 256) topk_range<8, 32>(A, t0, t1, f);
+    else if (A.E <= 512) topk_range<16, 32>(A, t0, t1, f);
+    else topk_range<32, 32>(A, t0, t1, f);
   }
 }
 
@@ -158,27 +182,6 @@ __device__ void scatter_pairs(const RouteArgs& A, int64_t p0, int64_t p1, const 
   }
 }
 
-__device__ __forceinline__ void topk_dispatch(const RouteArgs& A, int t0, int t1, int* s_cnt) {
-  if (A.E <= 32) topk_tokens<1>(A, t0, t1, s_cnt);
-  else if (A.E <= 64) topk_tokens<2>(A, t0, t1, s_cnt);
-  else if (A.E <= 128) topk_tokens<4>(A, t0, t1, s_cnt);
-  else if (A.E <= 256) topk_tokens<8>(A, t0, t1, s_cnt);
-  else if (A.E <= 512) topk_tokens<16>(A, t0, t1, s_cnt);
-  else topk_tokens<32>(A, t0, t1, s_cnt);
-}
-
-template <int PL>
-__device__ void fused_topk(const RouteArgs& A, int* s_ids, uint32_t* s_mask, int W) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  for (int t = warp; t < A.T; t += nwarps) {
-    const int e = topk_token<PL>(A, t);
-    if (lane < A.k) {
-      s_ids[t * A.k + lane] = e;
-      atomicOr(&s_mask[e * W + (t >> 5)], 1u << (t & 31));
-    }
-  }
-}
-
 // One CTA does everything (T <= kFusedMaxT).  A token picks an expert at most once, so the
 // tokens routed to expert e form a T-bit mask, and the rank of pair (t, j) among expert e's
 // pairs -- ordered by pair id, i.e. by token -- is the number of mask bits below t:
@@ -195,12 +198,10 @@ __global__ void __launch_bounds__(kFusedWarps * 32) route_fused_kernel(RouteArgs
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < A.E * W; i += blockDim.x) s_mask[i] = 0u;
   __syncthreads();
-  if (A.E <= 32) fused_topk<1>(A, s_ids, s_mask, W);
-  else if (A.E <= 64) fused_topk<2>(A, s_ids, s_mask, W);
-  else if (A.E <= 128) fused_topk<4>(A, s_ids, s_mask, W);
-  else if (A.E <= 256) fused_topk<8>(A, s_ids, s_mask, W);
-  else if (A.E <= 512) fused_topk<16>(A, s_ids, s_mask, W);
-  else fused_topk<32>(A, s_ids, s_mask, W);
+  topk_dispatch(A, 0, A.T, [&](int t, int e, int gl) {
+    s_ids[t * A.k + gl] = e;
+    atomicOr(&s_mask[e * W + (t >> 5)], 1u << (t & 31));
+  });
   __syncthreads();
   // exclusive scan of the per-expert counts (E <= blockDim.x)
   const int e = threadIdx.x;
@@ -253,7 +254,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(RouteArgs 
   __syncthreads();
   const int t0 = blockIdx.x * A.tokens_per_cta;
   const int t1 = min(A.T, t0 + A.tokens_per_cta);
-  topk_dispatch(A, t0, t1, s_cnt);
+  topk_dispatch(A, t0, t1, [&](int, int e, int) { atomicAdd(&s_cnt[e], 1); });
   __syncthreads();
   for (int e = threadIdx.x; e < A.E; e += blockDim.x) A.hist[blockIdx.x * A.E + e] = s_cnt[e];
 }

@@ -76,7 +76,8 @@ constexpr int kQPitch = kQBlock + 16;         // bytes per row pair in a stage's
 constexpr int kCodeBytes = kBN * kGS * 16;    // 16 KB
 constexpr int kBlockMaxKg = 24;               // scale-block mode: two 64-row blocks of <= 24 groups
 constexpr int kEpPitch = kBN + 4;             // floats per token row in the epilogue buffer
-constexpr int kDescBytes = 32;                // stage descriptor
+constexpr int kDescBytes = 16;                // stage descriptor
+constexpr int kPB = 12;                       // preparation pass: 256-k blocks per register batch
 // dynamic shared memory of the CTA (227 KB opt-in limit per block)
 constexpr int kSmemPerCta = 232448;
 
@@ -124,10 +125,18 @@ struct Unit {
 // Stage descriptor written by the producer next to the stage's data, read by the compute warps
 // after the stage's full barrier: the unit the stage belongs to and where it sits in it.
 enum : int { kDescFirst = 1, kDescLast = 2, kDescDone = 4 };
-struct StageDesc {
-  int r0, mt, g, flags;
-  int nt, e, g1, sp;
+// One 16-byte load: {r0, first group, tile, mt | groups << 5 | flags << 9 | x << 12} where x is
+// the expert (no split-K) or the K split (split-K runs on one expert).
+struct __align__(16) StageDesc {
+  int r0;
+  int g;
+  int nt;
+  int bits;
 };
+__device__ __forceinline__ int desc_mt(const StageDesc& d) { return d.bits & 31; }
+__device__ __forceinline__ int desc_gc(const StageDesc& d) { return (d.bits >> 5) & 15; }
+__device__ __forceinline__ int desc_flags(const StageDesc& d) { return (d.bits >> 9) & 7; }
+__device__ __forceinline__ int desc_x(const StageDesc& d) { return d.bits >> 12; }
 
 // Unit u -> (expert, token block, tile, split); `table` and `offs` live in shared memory.
 template <int MT>
@@ -175,17 +184,18 @@ __device__ __forceinline__ bool tile_row_valid(const StreamArgs& A, int nt, int 
 // fields at bits 0..3 / 16..19 as 1024 + u, at bits 4..7 / 20..23 as 1024 + 16 u -- times the
 // activation pair (b0, b1), plus c.  The extraction sits in the same asm block as the MMA so the
 // fragment registers live only across it.
+// The exponent pattern 0x64006400 comes in as a register (one immediate per lop3).
 __device__ __forceinline__ void mma_nib(float (&d)[4], uint32_t wl, uint32_t wh, uint32_t b0, uint32_t b1,
-                                        const float (&c)[4]) {
+                                        const float (&c)[4], uint32_t e1024) {
   asm("{\n .reg .b32 a0, a1, a2, a3;\n"
-      " lop3.b32 a0, %4, 0x000F000F, 0x64006400, 0xEA;\n"
-      " lop3.b32 a1, %5, 0x000F000F, 0x64006400, 0xEA;\n"
-      " lop3.b32 a2, %4, 0x00F000F0, 0x64006400, 0xEA;\n"
-      " lop3.b32 a3, %5, 0x00F000F0, 0x64006400, 0xEA;\n"
+      " lop3.b32 a0, %4, 0x000F000F, %12, 0xEA;\n"
+      " lop3.b32 a1, %5, 0x000F000F, %12, 0xEA;\n"
+      " lop3.b32 a2, %4, 0x00F000F0, %12, 0xEA;\n"
+      " lop3.b32 a3, %5, 0x00F000F0, %12, 0xEA;\n"
       " mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {a0,a1,a2,a3}, {%6,%7},"
       " {%8,%9,%10,%11};\n}\n"
       : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-      : "r"(wl), "r"(wh), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]), "f"(c[3]));
+      : "r"(wl), "r"(wh), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]), "f"(c[3]), "r"(e1024));
 }
 
 template <int MT, bool GELU, int SCALE>
@@ -300,13 +310,10 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         if (lane == 0) {
           StageDesc dsc;
           dsc.r0 = static_cast<int>(U.r0);
-          dsc.mt = U.mt;
           dsc.g = g;
-          dsc.flags = (g == U.g0 ? kDescFirst : 0) | (g + kGS >= U.g1 ? kDescLast : 0);
           dsc.nt = U.nt;
-          dsc.e = U.e;
-          dsc.g1 = U.g1;
-          dsc.sp = U.sp;
+          const int fl = (g == U.g0 ? kDescFirst : 0) | (g + kGS >= U.g1 ? kDescLast : 0);
+          dsc.bits = U.mt | (min(kGS, U.g1 - g) << 5) | (fl << 9) | ((A.splits > 1 ? U.sp : U.e) << 12);
           desc[slot] = dsc;
           uint32_t sbytes = 0;
           if (SCALE == kScaleTma) sbytes = 2 * kHalf * kGS * 2;
@@ -338,7 +345,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     if (!claim()) return;
     if (lane == 0) {
       StageDesc dsc{};
-      dsc.flags = kDescDone;
+      dsc.bits = kDescDone << 9;
       desc[slot] = dsc;
       mbar_arrive(&full[slot]);
     }
@@ -380,15 +387,17 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     const int slot = cslot;
     const uint32_t phase = cphase;
     if (++cslot == S) { cslot = 0; cphase ^= 1u; }
-    if (!mbar_wait(&full[slot], phase) || flags[0]) {
+    // (a producer that gave up leaves its stage incomplete: this bounded wait then ends the warp)
+    if (!mbar_wait(&full[slot], phase)) {
       if (lane == 0) { set_status(A.dev_status, W4_ERR_TIMEOUT); flags[0] = 1; }
       return;
     }
     const StageDesc dsc = desc[slot];
-    if (dsc.flags & kDescDone) return;
+    const int dflags = desc_flags(dsc);
+    if (dflags & kDescDone) return;
     const int g = dsc.g;
-    const int gc = min(kGS, dsc.g1 - g);
-    const int mt = dsc.mt;
+    const int gc = desc_gc(dsc);
+    const int mt = desc_mt(dsc);
     const uint8_t* xs = smem + L.x_off + slot * L.x_bytes;
     const uint8_t* qs = smem + L.q_off + slot * L.q_bytes;
     const uint8_t* ss = smem + L.sc_off + slot * L.sc_bytes;
@@ -409,15 +418,16 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         shi[p] = 2 * p < gc ? phi[p] : 0u;
       }
     } else {
-      const int64_t grow_lo = tile_row_valid(A, dsc.nt, rlo) ? tile_row(A, dsc.e, dsc.nt, rlo) : tile_row(A, dsc.e, dsc.nt, 0);
-      const int64_t grow_hi = tile_row_valid(A, dsc.nt, rhi) ? tile_row(A, dsc.e, dsc.nt, rhi) : tile_row(A, dsc.e, dsc.nt, 0);
+      const int dnt = dsc.nt, de = A.splits > 1 ? 0 : desc_x(dsc);
+      const int64_t grow_lo = tile_row_valid(A, dnt, rlo) ? tile_row(A, de, dnt, rlo) : tile_row(A, de, dnt, 0);
+      const int64_t grow_hi = tile_row_valid(A, dnt, rhi) ? tile_row(A, de, dnt, rhi) : tile_row(A, de, dnt, 0);
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         const int ga = g + 2 * p, gb = g + 2 * p + 1;
-        const uint32_t l0 = ga < dsc.g1 ? ldg_u16(A.scales + grow_lo * A.kg + ga) : 0;
-        const uint32_t l1 = gb < dsc.g1 ? ldg_u16(A.scales + grow_lo * A.kg + gb) : 0;
-        const uint32_t h0 = ga < dsc.g1 ? ldg_u16(A.scales + grow_hi * A.kg + ga) : 0;
-        const uint32_t h1 = gb < dsc.g1 ? ldg_u16(A.scales + grow_hi * A.kg + gb) : 0;
+        const uint32_t l0 = 2 * p < gc ? ldg_u16(A.scales + grow_lo * A.kg + ga) : 0;
+        const uint32_t l1 = 2 * p + 1 < gc ? ldg_u16(A.scales + grow_lo * A.kg + gb) : 0;
+        const uint32_t h0 = 2 * p < gc ? ldg_u16(A.scales + grow_hi * A.kg + ga) : 0;
+        const uint32_t h1 = 2 * p + 1 < gc ? ldg_u16(A.scales + grow_hi * A.kg + gb) : 0;
         slo[p] = l0 | (l1 << 16);
         shi[p] = h0 | (h1 << 16);
       }
@@ -434,6 +444,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       // one token block: extraction fused into the MMAs
       const uint8_t* xrow = xs + gid * kXPitch + tq * 16;
       const uint8_t* qrow = qs + tq * kQPitch;      // row pair (2tq, 2tq + 1)
+      const uint32_t e1024 = 0x64006400u;
 #pragma unroll
       for (int gi = 0; gi < kGS; ++gi) {
         const uint32_t aw = abase ^ static_cast<uint32_t>(gi << 4);
@@ -443,8 +454,8 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         const float4 cq = *reinterpret_cast<const float4*>(qrow + gi * 16);
         const float c[4] = {cq.x, cq.y, cq.z, cq.w};
         float d[4];
-        mma_nib(d, wlo, whi, xv.x, xv.y, c);
-        mma_nib(d, wlo >> 8, whi >> 8, xv.z, xv.w, d);
+        mma_nib(d, wlo, whi, xv.x, xv.y, c, e1024);
+        mma_nib(d, wlo >> 8, whi >> 8, xv.z, xv.w, d, e1024);
         const uint32_t sl = (gi & 1) ? (slo[gi >> 1] & 0xFFFF0000u) : (slo[gi >> 1] << 16);
         const uint32_t sh = (gi & 1) ? (shi[gi >> 1] & 0xFFFF0000u) : (shi[gi >> 1] << 16);
         acc[0][0] = fmaf(__uint_as_float(sl), d[0], acc[0][0]);
@@ -504,7 +515,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         }
       }
     }
-    const bool last = dsc.flags & kDescLast;
+    const bool last = dflags & kDescLast;
     if (last) {
       // undo the activation rows' power-of-two exponents (token columns 2tq, 2tq + 1 of each
       // block; the multipliers travel with the rows, so no global load waits behind the stream)
@@ -568,7 +579,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         for (int idx = ctid; idx < mt * kBN; idx += kWarps * 32) {
           const int t = idx / kBN, c = idx % kBN;
           if (n0 + c < A.N)
-            A.partial[(static_cast<int64_t>(dsc.sp) * A.rows + r0 + t) * A.N + n0 + c] = ep[t * kEpPitch + c];
+            A.partial[(static_cast<int64_t>(desc_x(dsc)) * A.rows + r0 + t) * A.N + n0 + c] = ep[t * kEpPitch + c];
         }
       }
       __threadfence();
@@ -631,51 +642,67 @@ stream_prep_kernel(const uint16_t* __restrict__ a, const int32_t* __restrict__ a
       }
     }
     const uint4* row = reinterpret_cast<const uint4*>(a + src * K);
+    // Lane l holds chunk l of up to kPB 256-k blocks at a time, all loads of a batch in flight
+    // together; a row of at most kPB blocks is read once.
+    uint4 v[kPB];
     uint32_t m = 0;
-    for (int i = lane; i < nv; i += 32) {
-      const uint4 v = __ldg(row + i);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int j0 = 0; j0 < nblk; j0 += kPB) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t lo = w[j] & 0x7FFFu, hi = (w[j] >> 16) & 0x7FFFu;
-        if (lo < 0x7F80u) m = max(m, lo);
-        if (hi < 0x7F80u) m = max(m, hi);
+      for (int t = 0; t < kPB; ++t) {
+        const int i = (j0 + t) * 32 + lane;
+        v[t] = i < nv ? __ldg(row + i) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int t = 0; t < kPB; ++t) {
+        const uint32_t w[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t lo = w[q] & 0x7FFFu, hi = (w[q] >> 16) & 0x7FFFu;
+          if (lo < 0x7F80u) m = max(m, lo);
+          if (hi < 0x7F80u) m = max(m, hi);
+        }
       }
     }
     m = __reduce_max_sync(0xffffffffu, m);
     const int f = shift_for(m, 14);
     const float m1 = pow2f(f), m16 = pow2f(f - 4);
     uint8_t* dst = xw + r * stride;
-    for (int j = 0; j < nblk; ++j) {
-      const int i = j * 32 + lane;
-      uint4 o = make_uint4(0, 0, 0, 0);
-      float part = 0.f;
-      if (i < nv) {
-        const uint4 v = __ldg(row + i);
-        const __half2 h0 = __floats2half2_rn(bf16_lo_to_f32(v.x) * m1, bf16_hi_to_f32(v.x) * m1);
-        const __half2 h1 = __floats2half2_rn(bf16_lo_to_f32(v.y) * m16, bf16_hi_to_f32(v.y) * m16);
-        const __half2 h2 = __floats2half2_rn(bf16_lo_to_f32(v.z) * m1, bf16_hi_to_f32(v.z) * m1);
-        const __half2 h3 = __floats2half2_rn(bf16_lo_to_f32(v.w) * m16, bf16_hi_to_f32(v.w) * m16);
+    for (int j0 = 0; j0 < nblk; j0 += kPB) {
+      if (nblk > kPB) {                          // long rows: the batch again (from L1 / L2)
+#pragma unroll
+        for (int t = 0; t < kPB; ++t) {
+          const int i = (j0 + t) * 32 + lane;
+          v[t] = i < nv ? __ldg(row + i) : make_uint4(0, 0, 0, 0);
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < kPB; ++t) {
+        const int j = j0 + t;
+        if (j >= nblk) break;
+        const __half2 h0 = __floats2half2_rn(bf16_lo_to_f32(v[t].x) * m1, bf16_hi_to_f32(v[t].x) * m1);
+        const __half2 h1 = __floats2half2_rn(bf16_lo_to_f32(v[t].y) * m16, bf16_hi_to_f32(v[t].y) * m16);
+        const __half2 h2 = __floats2half2_rn(bf16_lo_to_f32(v[t].z) * m1, bf16_hi_to_f32(v[t].z) * m1);
+        const __half2 h3 = __floats2half2_rn(bf16_lo_to_f32(v[t].w) * m16, bf16_hi_to_f32(v[t].w) * m16);
         const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
         const float2 f2 = __half22float2(h2), f3 = __half22float2(h3);
-        part = 1032.f * ((f0.x + f0.y) + (f2.x + f2.y)) + 1152.f * ((f1.x + f1.y) + (f3.x + f3.y));
-        o = make_uint4(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1),
-                       *reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&h3));
-      }
-      uint8_t* blk = dst + static_cast<int64_t>(j) * kPrepStage;
-      *reinterpret_cast<uint4*>(blk + lane * 16) = o;
-      part += __shfl_xor_sync(0xffffffffu, part, 1);
-      part += __shfl_xor_sync(0xffffffffu, part, 2);
-      if ((lane & 3) == 0) {
-        const float c = -part;
-        float* q = reinterpret_cast<float*>(blk + kXCopy + (lane >> 2) * 16);
-        q[0] = c;
-        q[2] = c;
-        if (r + 1 == rows) { q[1] = 0.f; q[3] = 0.f; }
-        if (r > 0) {
-          float* qp = reinterpret_cast<float*>(blk - stride + kXCopy + (lane >> 2) * 16);
-          qp[1] = c;
-          qp[3] = c;
+        float part = 1032.f * ((f0.x + f0.y) + (f2.x + f2.y)) + 1152.f * ((f1.x + f1.y) + (f3.x + f3.y));
+        const uint4 o = make_uint4(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1),
+                                   *reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&h3));
+        uint8_t* blk = dst + static_cast<int64_t>(j) * kPrepStage;
+        *reinterpret_cast<uint4*>(blk + lane * 16) = o;
+        part += __shfl_xor_sync(0xffffffffu, part, 1);
+        part += __shfl_xor_sync(0xffffffffu, part, 2);
+        if ((lane & 3) == 0) {
+          const float c = -part;
+          float* q = reinterpret_cast<float*>(blk + kXCopy + (lane >> 2) * 16);
+          q[0] = c;
+          q[2] = c;
+          if (r + 1 == rows) { q[1] = 0.f; q[3] = 0.f; }
+          if (r > 0) {
+            float* qp = reinterpret_cast<float*>(blk - stride + kXCopy + (lane >> 2) * 16);
+            qp[1] = c;
+            qp[3] = c;
+          }
         }
       }
     }
