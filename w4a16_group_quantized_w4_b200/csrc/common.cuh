@@ -75,6 +75,28 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// try_wait without a suspend-time hint (the hardware's own time limit per try)
+__device__ __forceinline__ bool mbar_try_wait_nohint(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+// Bounded wait of the streaming kernel's rings (no suspend hint: a waiting warp resumes sooner
+// once the phase completes); returns false once kWaitLimitNs have passed.
+__device__ __forceinline__ bool mbar_wait_ring(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait_nohint(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_nohint(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
 // Bounded wait: returns false once kWaitLimitNs have passed (the caller reports W4_ERR_TIMEOUT).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;

@@ -286,7 +286,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     auto claim = [&]() -> bool {
       if (!first_lap) {
         bool ok = true;
-        if (lane == 0) ok = mbar_wait(&empty[slot], phase);
+        if (lane == 0) ok = mbar_wait_ring(&empty[slot], phase);
         if (!__shfl_sync(0xffffffffu, ok, 0) || flags[0]) {
           if (lane == 0) { set_status(A.dev_status, W4_ERR_TIMEOUT); flags[0] = 1; }
           return false;
@@ -388,7 +388,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     const uint32_t phase = cphase;
     if (++cslot == S) { cslot = 0; cphase ^= 1u; }
     // (a producer that gave up leaves its stage incomplete: this bounded wait then ends the warp)
-    if (!mbar_wait(&full[slot], phase)) {
+    if (!mbar_wait_ring(&full[slot], phase)) {
       if (lane == 0) { set_status(A.dev_status, W4_ERR_TIMEOUT); flags[0] = 1; }
       return;
     }
@@ -600,9 +600,17 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         for (int idx = ctid; idx < mt * kBN; idx += kWarps * 32) {
           const int t = idx / kBN, c = idx % kBN;
           if (n0 + c < A.N) {
+            // the partials of up to 8 splits are loaded together, then summed in split order
+            const float* pp = A.partial + (r0 + t) * A.N + n0 + c;
+            const int64_t ps = A.rows * A.N;
             float sum = 0.f;
-            for (int sp = 0; sp < A.splits; ++sp)
-              sum += __ldcg(&A.partial[(static_cast<int64_t>(sp) * A.rows + r0 + t) * A.N + n0 + c]);
+            for (int sp0 = 0; sp0 < A.splits; sp0 += 8) {
+              float pv[8];
+#pragma unroll
+              for (int q = 0; q < 8; ++q) pv[q] = sp0 + q < A.splits ? __ldcg(pp + (sp0 + q) * ps) : 0.f;
+#pragma unroll
+              for (int q = 0; q < 8; ++q) sum += pv[q];
+            }
             A.out[(r0 + t) * A.N + n0 + c] = f32_to_bf16_bits(sum);
           }
         }
@@ -810,11 +818,12 @@ static StreamPlan plan_stream(int64_t rows, int N, int K, int E, int epi, bool d
                                         : (N + w4::kBN - 1) / w4::kBN;
   p.splits = 1;
   if (dense) {
-    // split K while the units do not fill the CTAs four times over and the float32 partials
-    // stay below ~1/8 of the weight bytes
+    // split K only while the units cover fewer than ~3/4 of the pipelines (long units stream
+    // better than many short ones: a K = 4096 GEMV measured fastest with two splits) and the
+    // float32 partials stay below ~1/8 of the weight bytes
     const int64_t ntb = (rows + p.MT - 1) / p.MT;
     const double wbytes = static_cast<double>(N) * K * 0.5625;
-    while (p.splits * 2 <= kstages && ntb * p.n_tiles * p.splits < 4LL * w4::kPipes * sm_count &&
+    while (p.splits * 2 <= kstages && 4 * ntb * p.n_tiles * p.splits < 3LL * w4::kPipes * sm_count &&
            static_cast<double>(p.splits * 2) * rows * N * 8.0 <= wbytes / 8.0)
       p.splits *= 2;
   }
