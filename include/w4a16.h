@@ -106,7 +106,8 @@ w4_status w4_repack(const uint16_t* w, int64_t rows, int64_t K, uint32_t* codes,
  * Two kernels serve the call: for M < 64 (or N % 128 != 0, or K > 4096, or K % 64 != 0) a
  * weight-streaming kernel (workspace: M * ceil(K/256) * 656 bytes of prepared rows -- fp16
  * values, the row multiplier and per-group bias corrections -- and split-K partials), otherwise the
- * tensor-core kernel (workspace: M * K * 2 bytes plus 4 per row).  In the streaming kernel each
+ * tensor-core kernel (workspace: M * K * 2 bytes and 4 per row, each rounded up to 256, plus one
+ * byte per weight row).  In the streaming kernel each
  * group's sum also carries a float32 rounding of a bias term that its correction cancels: about
  * 2^-13 of the group's mean |x| times 32 per group, far below the bf16 output rounding.
  */
@@ -153,8 +154,9 @@ w4_status moe_route_permute(const float* logits, int32_t T, int32_t E, int32_t k
  *                   (W4_ERR_WORKSPACE when smaller; nonzero whenever rows > 0): every sorted row
  *                   of `a` written once, in sorted order, in fp16 with a power-of-two exponent.
  *                   The tensor-core kernel (rows >= 32 * E, K <= 4096, K % 64 == 0, N % 128 == 0
- *                   or (N/2) % 64 == 0 with W4_EPI_GELU_GATE) needs rows * K * 2 bytes plus 4
- *                   per row; the weight-streaming kernel rows * ceil(K/256) * 656 bytes (fp16
+ *                   or (N/2) % 64 == 0 with W4_EPI_GELU_GATE) needs rows * K * 2 bytes and 4
+ *                   per row (each rounded up to 256) plus E * N bytes (a power-of-two exponent per
+ *                   weight row); the weight-streaming kernel rows * ceil(K/256) * 656 bytes (fp16
  *                   values, the row multiplier and per-group bias corrections).
  *   dev_status      one int32 device word or NULL: set to a w4_status code if the device finds a
  *                   problem (offsets out of range: W4_ERR_INVALID_ARG; a pair naming a row past

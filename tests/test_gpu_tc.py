@@ -18,14 +18,15 @@ from tests._util import assert_rows_close, dev_bf16, dev_f32, dev_u32, host_f64
 pytestmark = pytest.mark.gpu
 
 
-def _tc_bytes(rows, K):
-    return (rows * K * 2 + 255) // 256 * 256 + rows * 4
+def _tc_bytes(rows, K, wrows):
+    """fp16 rows and row multipliers (each 256-byte aligned), then one exponent byte per weight row."""
+    return (rows * K * 2 + 255) // 256 * 256 + (rows * 4 + 255) // 256 * 256 + wrows
 
 
 @pytest.mark.parametrize("M,N,K", [(64, 128, 64), (128, 128, 256), (200, 384, 512),
                                    (513, 128, 2816), (130, 256, 4096), (1000, 1408 * 2, 704)])
 def test_dense_tc_shapes(M, N, K):
-    assert api.w4_workspace_bytes(_lib.W4_OP_LINEAR, M, N, K, 1, 1) == _tc_bytes(M, K)
+    assert api.w4_workspace_bytes(_lib.W4_OP_LINEAR, M, N, K, 1, 1) == _tc_bytes(M, K, N)
     case = synth.dense_case(M, N, K, 0.02, 1e-3, seed=M + 3 * N + K)
     y = api.w4a16_linear(dev_bf16(case.x), dev_u32(case.codes), dev_bf16(case.scales))
     torch.cuda.synchronize()
@@ -65,7 +66,7 @@ def _route(logits, k):
                                             (300, 4, 2, 128, 64, None)])
 def test_grouped_tc_gate_up_and_down(T, E, k, H, I, zipf):
     case = synth.moe_case(T, E, k, H, I, seed=T + E, zipf_s=zipf)
-    assert api.w4_workspace_bytes(_lib.W4_OP_GMM, T * k, 2 * I, H, E, k) == _tc_bytes(T * k, H)
+    assert api.w4_workspace_bytes(_lib.W4_OP_GMM, T * k, 2 * I, H, E, k) == _tc_bytes(T * k, H, E * 2 * I)
     rt = _route(case.logits, k)
     ref_rt = moe.route(case.logits, k)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")

@@ -22,7 +22,7 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
                                 const int32_t* offsets, int E, int64_t rows, int N, int K, int epi,
                                 uint16_t* out, void* ws, size_t ws_bytes, int32_t* dev_status,
                                 cudaStream_t stream, int sm_count);
-size_t w4_tc_workspace_bytes(int64_t rows, int K);
+size_t w4_tc_workspace_bytes(int64_t rows, int K, int64_t wrows);
 bool w4_tm_supported(int N, int K, int epi);
 w4_status w4_launch_tm_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int k_div,
                             const uint32_t* codes, const uint16_t* scales, const int32_t* offsets,
@@ -90,7 +90,7 @@ size_t w4_workspace_bytes(int32_t op, int64_t M_or_T, int64_t N, int64_t K, int3
     case W4_OP_LINEAR:
       if (N <= 0 || K < 32 || K % 32) return 0;
       if (use_tc(M_or_T, 1, static_cast<int>(N), static_cast<int>(K), W4_EPI_NONE, true, nullptr))
-        return w4_tc_workspace_bytes(M_or_T, static_cast<int>(K));
+        return w4_tc_workspace_bytes(M_or_T, static_cast<int>(K), N);
       return w4_stream_workspace_bytes(M_or_T, static_cast<int>(N), static_cast<int>(K), 1,
                                        W4_EPI_NONE, true, current_sm_count());
     case W4_OP_ROUTE:
@@ -102,7 +102,7 @@ size_t w4_workspace_bytes(int32_t op, int64_t M_or_T, int64_t N, int64_t K, int3
       size_t need = 0;
       for (int epi : {W4_EPI_NONE, W4_EPI_GELU_GATE}) {
         const size_t b = use_tc(M_or_T, E, static_cast<int>(N), static_cast<int>(K), epi, false, nullptr)
-                             ? w4_tc_workspace_bytes(M_or_T, static_cast<int>(K))
+                             ? w4_tc_workspace_bytes(M_or_T, static_cast<int>(K), static_cast<int64_t>(E) * N)
                              : w4_stream_workspace_bytes(M_or_T, static_cast<int>(N), static_cast<int>(K), E,
                                                          epi, false, current_sm_count());
         if (b > need) need = b;

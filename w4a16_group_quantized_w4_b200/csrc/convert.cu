@@ -65,29 +65,60 @@ a_to_f16_kernel(const uint16_t* __restrict__ a, const int32_t* __restrict__ a_ro
   }
 }
 
+// Per weight row (one thread each): the exponent e that brings the row's largest finite scale
+// to [2^10, 2^11), as in the dequantisation of tm_gemm.cu.  Rows of kg bf16 scales, kg even (4-byte
+// aligned words).
+__global__ void __launch_bounds__(256)
+row_exp_kernel(const uint16_t* __restrict__ scales, int64_t wrows, int kg, int8_t* __restrict__ e_out) {
+  for (int64_t r = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; r < wrows;
+       r += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint32_t* row = reinterpret_cast<const uint32_t*>(scales + r * kg);
+    uint32_t m = 0;
+    for (int j = 0; j < (kg >> 1); ++j) {
+      const uint32_t v = __ldg(row + j);
+      const uint32_t lo = v & 0x7FFFu, hi = (v >> 16) & 0x7FFFu;
+      if (lo < 0x7F80u) m = max(m, lo);
+      if (hi < 0x7F80u) m = max(m, hi);
+    }
+    e_out[r] = static_cast<int8_t>(shift_for(m, 10));
+  }
+}
+
 }  // namespace cv
 }  // namespace w4
 
 // fp16 activation rows in pair order [rows, K] (256-byte aligned), then the row multipliers
-size_t w4_tc_workspace_bytes(int64_t rows, int K) {
+// [rows] (256-byte aligned), then the weight-row exponents [wrows] (int8)
+static size_t a16_bytes(int64_t rows, int K) { return (static_cast<size_t>(rows) * K * 2 + 255) / 256 * 256; }
+static size_t rowmul_bytes(int64_t rows) { return (static_cast<size_t>(rows) * 4 + 255) / 256 * 256; }
+
+size_t w4_tc_workspace_bytes(int64_t rows, int K, int64_t wrows) {
   if (rows <= 0) return 0;
-  return (static_cast<size_t>(rows) * K * 2 + 255) / 256 * 256 + static_cast<size_t>(rows) * 4;
+  return a16_bytes(rows, K) + rowmul_bytes(rows) + static_cast<size_t>(wrows);
 }
 
 uint16_t* w4_ws_a16(void* ws) { return static_cast<uint16_t*>(ws); }
 
 float* w4_ws_rowmul(void* ws, int64_t rows, int K) {
-  return reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
-                                  (static_cast<size_t>(rows) * K * 2 + 255) / 256 * 256);
+  return reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + a16_bytes(rows, K));
+}
+
+int8_t* w4_ws_rowexp(void* ws, int64_t rows, int K) {
+  return reinterpret_cast<int8_t*>(static_cast<uint8_t*>(ws) + a16_bytes(rows, K) + rowmul_bytes(rows));
 }
 
 void w4_launch_a_to_f16(const uint16_t* a, const int32_t* a_row_of_pair, int k_div, int64_t a_rows,
-                        int64_t rows, int K, void* ws, int32_t* dev_status, cudaStream_t stream,
-                        int sm_count) {
+                        int64_t rows, int K, const uint16_t* scales, int64_t wrows, void* ws,
+                        int32_t* dev_status, cudaStream_t stream, int sm_count) {
   if (rows <= 0) return;
   const int64_t blocks = (rows + 7) / 8;
   const int grid = static_cast<int>(blocks < 16LL * sm_count ? blocks : 16LL * sm_count);
   w4::cv::a_to_f16_kernel<<<grid, 256, 0, stream>>>(a, a_row_of_pair, k_div, a_rows, rows, K,
                                                     w4_ws_a16(ws), w4_ws_rowmul(ws, rows, K),
                                                     dev_status);
+  if (wrows > 0) {
+    const int64_t eb = (wrows + 255) / 256;
+    const int egrid = static_cast<int>(eb < 8LL * sm_count ? eb : 8LL * sm_count);
+    w4::cv::row_exp_kernel<<<egrid, 256, 0, stream>>>(scales, wrows, K / 32, w4_ws_rowexp(ws, rows, K));
+  }
 }

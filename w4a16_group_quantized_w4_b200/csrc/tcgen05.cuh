@@ -118,10 +118,13 @@ __device__ __forceinline__ void tmem_wait_st() {
 // Conversion pass in front of the tensor-core kernels (convert.cu): row p of a16 becomes the
 // activation row that routed row p reads (row p of `a`, or a_row_of_pair[p] / k_div), as
 // fp16(a * 2^f) with f picked from the row's largest finite magnitude, and rowmul[p] = 2^-f.
-size_t w4_tc_workspace_bytes(int64_t rows, int K);
+// The same launch also writes, per weight row (wrows = E * N rows of kg scales), the power-of-two
+// exponent e that brings the row's largest finite scale to [2^10, 2^11) (int8).
+size_t w4_tc_workspace_bytes(int64_t rows, int K, int64_t wrows);
 void w4_launch_a_to_f16(const uint16_t* a, const int32_t* a_row_of_pair, int k_div, int64_t a_rows,
-                        int64_t rows, int K, void* ws, int32_t* dev_status, cudaStream_t stream,
-                        int sm_count);
+                        int64_t rows, int K, const uint16_t* scales, int64_t wrows, void* ws,
+                        int32_t* dev_status, cudaStream_t stream, int sm_count);
 // pointers into a workspace laid out by w4_tc_workspace_bytes
 uint16_t* w4_ws_a16(void* ws);
 float* w4_ws_rowmul(void* ws, int64_t rows, int K);
+int8_t* w4_ws_rowexp(void* ws, int64_t rows, int K);

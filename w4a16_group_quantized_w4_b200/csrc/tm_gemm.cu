@@ -43,9 +43,13 @@
 //   warp 3       token producer: per stage, 2-D TMA boxes of 64 k x NMAX rows (128-byte swizzle)
 //   warp 1       TMEM allocation and the MMA-issuing thread (warps 16.. add issuers when the
 //                configuration splits a tile's MMAs over several threads)
-//   warp 2       per tile, the scale block by cp.async into bank-padded rows
+//   warp 2       idle (the dequant warps read their scales from global memory, see below)
 //   warps 4-7    epilogue: tcgen05.ld of the accumulator, exponents, GELU gate, bf16 stores
-//   warps 8-15   dequant: codes + scales -> fp16 pairs -> tcgen05.st into the TMEM A slots
+//   warps 8-15   dequant: codes + scales -> fp16 pairs -> tcgen05.st into the TMEM A slots.
+//                Each thread owns one weight row: its exponent e comes from the conversion pass
+//                (one byte per weight row, loaded a tile ahead) and its two scales per stage
+//                straight from global memory through a three-stage register queue that runs
+//                ahead across tiles, so no shared memory is spent on scale blocks.
 // Every wait is bounded (W4_ERR_TIMEOUT in dev_status instead of a hang).
 #include <cudaTypedefs.h>
 
@@ -66,7 +70,6 @@ constexpr int kACols = 64;                               // TMEM columns per A s
 struct Lay {
   int code;                 // code ring: cst stages
   int cst;
-  int sc, scb;              // two scale blocks of scb bytes (rows padded to an odd word count)
   int sh;                   // float [2][128]: 2^-e per TMEM lane
   int bars;
   int tmem_slot;            // + abort flag
@@ -76,6 +79,7 @@ struct Lay {
 
 struct Args {
   const float* rowmul;      // [rows] 2^-f of each converted activation row
+  const int8_t* rowexp;     // [E*N] exponent e of each weight row
   const uint16_t* scales;   // [E*N, kg]
   const int32_t* offsets;   // [E+1] or null (dense: one expert with `rows` rows)
   int E, N, K, kg, nst;     // nst = stages per tile
@@ -123,8 +127,8 @@ struct Cfg {
   static constexpr int tok = 0;                          // token ring at the base
   static constexpr int code = TSTAGES * kTokStage;       // code ring after it
   // cfull, cfree (x kMaxCStages), tfull, tfree (x TSTAGES), a_ready, a_free (x ASLOTS),
-  // acc_full, acc_empty, sc_full, sc_empty, sh_full, sh_empty (x 2)
-  static constexpr int nbars = 2 * kMaxCStages + 2 * TSTAGES + 2 * ASLOTS + 12;
+  // acc_full, acc_empty, sh_full, sh_empty (x 2)
+  static constexpr int nbars = 2 * kMaxCStages + 2 * TSTAGES + 2 * ASLOTS + 8;
   static_assert(kTokSub % 1024 == 0, "128-byte swizzle atoms");
 };
 
@@ -220,9 +224,7 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
   uint64_t* a_free = a_ready + ASLOTS;
   uint64_t* acc_full = a_free + ASLOTS;
   uint64_t* acc_empty = acc_full + 2;
-  uint64_t* sc_full = acc_empty + 2;
-  uint64_t* sc_empty = sc_full + 2;
-  uint64_t* sh_full = sc_empty + 2;
+  uint64_t* sh_full = acc_empty + 2;
   uint64_t* sh_empty = sh_full + 2;
   float* sh = reinterpret_cast<float*>(smem + L.sh);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.tmem_slot);
@@ -277,8 +279,6 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], C::kIssuers);
       mbar_init(&acc_empty[b], C::kEpiWarps);
-      mbar_init(&sc_full[b], 32);    // the scale loader's lanes (cp.async arrivals)
-      mbar_init(&sc_empty[b], 8);
       mbar_init(&sh_full[b], 4);     // the dequant warps of the first k half
       mbar_init(&sh_empty[b], C::kEpiWarps);
     }
@@ -405,30 +405,6 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       if (!ok) fail(0);
     }
     __syncwarp();
-  } else if (warp == 2) {
-    // ------------------------------ scale loader ------------------------------
-    const int hw = A.kg >> 1;                 // words per row in global memory
-    const int P = hw | 1;                     // words per row in shared memory (odd)
-    int ti = 0;
-    for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x, ++ti) {
-      Tile T;
-      decode_tile(A, table, offs, t, NMAX, T);
-      const int sb = ti & 1;
-      if (ti >= 2 && !mbar_wait(&sc_empty[sb], ((ti >> 1) - 1) & 1)) { fail(lane); break; }
-      const uint32_t dst0 = smem_u32(smem + L.sc + sb * L.scb);
-      const uint32_t* src_a = reinterpret_cast<const uint32_t*>(A.scales + wrow(A, T, 0) * A.kg);
-      const uint32_t* src_b = reinterpret_cast<const uint32_t*>(A.scales + wrow(A, T, kBM / 2) * A.kg);
-      for (int w = lane; w < kBM * hw; w += 32) {
-        const int rr = w / hw, j = w - rr * hw;
-        const uint32_t* src = rr < kBM / 2 ? src_a + w : src_b + (w - (kBM / 2) * hw);
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;"
-                     ::"r"(dst0 + (rr * P + j) * 4), "l"(src) : "memory");
-      }
-      // each lane's arrival lands once its copies have
-      asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&sc_full[sb]))
-                   : "memory");
-    }
-    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if ((warp >= 4 && warp < 8) || warp >= C::kEpiWarp1) {
     // ------------------------------ epilogue ------------------------------
     // TMEM lanes 32q .. 32q+31 are readable by warps with warp % 4 == q; with two epilogue warps
@@ -460,12 +436,21 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] += w[i];
         }
+        // the 16 token rows' multipliers: four 16-byte loads when the chunk is whole and aligned
+        float rm[16];
+        const float* rp = A.rowmul + T.r0 + c0;
+        if (c0 + 16 <= T.mrows && (reinterpret_cast<uintptr_t>(rp) & 15) == 0) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int tk = c0 + i;
-          const float rm = tk < T.mrows ? __ldg(A.rowmul + T.r0 + tk) : 0.f;
-          v[i] = (v[i] * rm) * cm;
+          for (int i = 0; i < 4; ++i) {
+            const float4 f = __ldg(reinterpret_cast<const float4*>(rp) + i);
+            rm[4 * i] = f.x; rm[4 * i + 1] = f.y; rm[4 * i + 2] = f.z; rm[4 * i + 3] = f.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) rm[i] = c0 + i < T.mrows ? __ldg(rp + i) : 0.f;
         }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = (v[i] * rm[i]) * cm;
         if (gelu) {
           // lanes i < 16: gate values, lanes i + 16: up values of the same output j; the lower
           // lane finishes tokens c0 .. c0+7, the upper one tokens c0+8 .. c0+15
@@ -506,8 +491,43 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     // swizzle phase of code row r: 64-byte swizzle XORs the 16-byte chunk with address bits 7-8
     // ((r >> 1) & 3 at a 64-byte pitch), 128-byte swizzle with bits 7-9 (r & 7 at a 128-byte pitch)
     const int sw = KSK == 128 ? ((r >> 1) & 3) : (r & 7);
-    const int P = (A.kg >> 1) | 1;
     const uint32_t tlane = static_cast<uint32_t>(q * 32) << 16;
+    // Scale queue: the word holding groups g0, g0 + 1 of this row for each (tile, stage, half) in
+    // order, kSQ entries ahead of the dequantisation, loaded from global memory (L2-resident
+    // after the first touch of a 32-byte sector), across tile boundaries.
+    constexpr int kSQ = 3;
+    uint32_t sq[kSQ];
+    int pf_t = blockIdx.x, pf_st = 0, pf_hf = 0;
+    const uint32_t* pf_row = nullptr;            // this thread's scale row in tile pf_t
+    auto pf_tile = [&]() {
+      if (pf_t < total) {
+        Tile P;
+        decode_tile(A, table, offs, pf_t, NMAX, P);
+        pf_row = reinterpret_cast<const uint32_t*>(A.scales + wrow(A, P, r) * A.kg);
+      }
+    };
+    auto pf_next = [&]() -> uint32_t {
+      uint32_t v = 0u;
+      if (pf_t < total) {
+        const int g0 = pf_st * (KSK / 32) + 4 * pf_hf + 2 * h;
+        if (g0 < A.kg) v = __ldg(pf_row + (g0 >> 1));     // groups past K: scale 0
+        if (++pf_hf == C::kHalves) {
+          pf_hf = 0;
+          if (++pf_st == nst) { pf_st = 0; pf_t += gridDim.x; pf_tile(); }
+        }
+      }
+      return v;
+    };
+    pf_tile();
+#pragma unroll
+    for (int i = 0; i < kSQ; ++i) sq[i] = pf_next();
+    // exponent of this row, one tile ahead
+    int e_next = 0;
+    if (blockIdx.x < static_cast<unsigned>(total)) {
+      Tile T0;
+      decode_tile(A, table, offs, blockIdx.x, NMAX, T0);
+      e_next = A.rowexp[wrow(A, T0, r)];
+    }
     int slot = 0, aslot = 0;
     uint32_t ph = 0, aph = 0;
     bool alap0 = true;
@@ -515,18 +535,14 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++ti) {
       const int sb = ti & 1;
-      if (!mbar_wait(&sc_full[sb], (ti >> 1) & 1)) { ok = false; break; }
-      const uint32_t* srow = reinterpret_cast<const uint32_t*>(smem + L.sc + sb * L.scb) + r * P;
-      // row exponent e: the row's largest finite |scale| lands in [2^10, 2^11), so 24 s' stays
-      // below 2^16 and every scale within 2^21 of the largest keeps s'' and 24 s' exact
-      uint32_t m = 0;
-      for (int j = 0; j < (A.kg >> 1); ++j) {
-        const uint32_t v = srow[j];
-        const uint32_t lo = v & 0x7FFFu, hi = (v >> 16) & 0x7FFFu;
-        if (lo < 0x7F80u) m = max(m, lo);
-        if (hi < 0x7F80u) m = max(m, hi);
+      const int e = e_next;
+      if (t + static_cast<int>(gridDim.x) < total) {
+        Tile Tn;
+        decode_tile(A, table, offs, t + gridDim.x, NMAX, Tn);
+        e_next = A.rowexp[wrow(A, Tn, r)];
       }
-      const int e = shift_for(m, 10);
+      // e brings the row's largest finite |scale| to [2^10, 2^11), so 24 s' stays below 2^16 and
+      // every scale within 2^21 of the largest keeps s'' and 24 s' exact
       const float smul = pow2f(e - 6);
       if (h == 0) {
         if (ti >= 2 && !mbar_wait(&sh_empty[sb], ((ti >> 1) - 1) & 1)) { ok = false; break; }
@@ -548,8 +564,10 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         if (++slot == cst) { slot = 0; ph ^= 1u; }
 #pragma unroll
         for (int hf = 0; hf < C::kHalves; ++hf) {
-          const int g0 = st * (KSK / 32) + 4 * hf + 2 * h;
-          const uint32_t sv = g0 < A.kg ? srow[g0 >> 1] : 0u;   // groups past K: scale 0
+          const uint32_t sv = sq[0];
+#pragma unroll
+          for (int i = 0; i + 1 < kSQ; ++i) sq[i] = sq[i + 1];
+          sq[kSQ - 1] = pf_next();
           uint32_t s2a, c2a, s2b, c2b;
           scale_pair(sv & 0xFFFFu, smul, s2a, c2a);
           scale_pair(sv >> 16, smul, s2b, c2b);
@@ -575,8 +593,6 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         if (!ok) break;
       }
       if (!ok) break;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sc_empty[sb]);
     }
     if (!ok) fail(lane);
   }
@@ -622,15 +638,14 @@ constexpr int kTmSmemBudget = 232448 - 1024;
 template <int NMAX, int KSK, int TSTAGES, int ASLOTS, int NSPLIT, int KSPLIT, int ABUF, int EPIW>
 static bool tm_layout(int E, int kg, w4::tm::Lay& L) {
   using C = w4::tm::Cfg<NMAX, KSK, TSTAGES, ASLOTS, NSPLIT, KSPLIT, ABUF, EPIW>;
+  (void)kg;
   L.code = C::code;
-  L.scb = (w4::tm::kBM * ((kg >> 1) | 1) * 4 + 127) / 128 * 128;
-  const int fixed = 2 * L.scb + 2 * w4::tm::kBM * 4 + C::nbars * 8 + 16 + (E + 1) * 8;
+  const int fixed = 2 * w4::tm::kBM * 4 + C::nbars * 8 + 16 + (E + 1) * 8;
   int cst = (kTmSmemBudget - L.code - fixed) / C::kCodeStage;
   if (cst > w4::tm::kMaxCStages) cst = w4::tm::kMaxCStages;
   if (cst < 2) return false;
   L.cst = cst;
-  L.sc = L.code + cst * C::kCodeStage;
-  L.sh = L.sc + 2 * L.scb;
+  L.sh = L.code + cst * C::kCodeStage;
   L.bars = L.sh + 2 * w4::tm::kBM * 4;
   L.tmem_slot = L.bars + C::nbars * 8;
   L.table = L.tmem_slot + 16;
@@ -697,20 +712,23 @@ w4_status w4_launch_tm_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int
   const int kd = k_div > 0 ? k_div : 1;
   const int64_t a_rows = a_row_of_pair ? rows / kd : rows;   // rows of `a` a pair may name
   if (a_rows <= 0) return W4_ERR_INVALID_ARG;
-  if (!ws || ws_bytes < w4_tc_workspace_bytes(rows, K) || (reinterpret_cast<uintptr_t>(ws) & 15))
+  const int64_t wrows = static_cast<int64_t>(E) * N;
+  if (!ws || ws_bytes < w4_tc_workspace_bytes(rows, K, wrows) || (reinterpret_cast<uintptr_t>(ws) & 15))
     return W4_ERR_WORKSPACE;
-  w4_launch_a_to_f16(a, a_row_of_pair, kd, a_rows, rows, K, ws, dev_status, stream, sm_count);
+  w4_launch_a_to_f16(a, a_row_of_pair, kd, a_rows, rows, K, scales, wrows, ws, dev_status, stream,
+                     sm_count);
 
   w4::tm::Args A{};
   A.rowmul = w4_ws_rowmul(ws, rows, K);
+  A.rowexp = w4_ws_rowexp(ws, rows, K);
   A.scales = scales; A.offsets = offsets;
   A.E = E; A.N = N; A.K = K; A.kg = K / 32;
   A.rows = rows; A.epi = epi; A.out = out;
   A.n_tiles = (epi == W4_EPI_GELU_GATE) ? (N / 2) / (w4::tm::kBM / 2) : N / w4::tm::kBM;
   A.dev_status = dev_status;
   const uint16_t* a16 = w4_ws_a16(ws);
-  // 256-row token blocks, 128-k stages, two MMA-issuing threads (128 token columns each, the
-  // tensor pipe's rate needs more than one issuer), one 256-column accumulator drained by eight
-  // epilogue warps
-  return tm_launch_cfg<192, 128, 2, 2, 2, 1, 2, 2>(codes, a16, rows, K, A, stream, sm_count);
+  // 192-row token blocks, 128-k stages with three token stages in flight, two MMA-issuing
+  // threads (96 token columns each: the tensor pipe's rate needs more than one issuer), two
+  // 192-column accumulators drained by eight epilogue warps
+  return tm_launch_cfg<192, 128, 3, 2, 2, 1, 2, 2>(codes, a16, rows, K, A, stream, sm_count);
 }
