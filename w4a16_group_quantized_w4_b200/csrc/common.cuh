@@ -207,8 +207,34 @@ __device__ __forceinline__ float gelu_tanh(float z) {
   return 0.5f * z * (1.0f + tanhf(c * (z + 0.044715f * z * z * z)));
 }
 
+// Programmatic dependent launch.  pdl_trigger lets the next kernel on the stream (launched with
+// launch_pdl) start launching while this one runs; pdl_wait blocks until the previous kernel on
+// the stream has completed and its memory operations are visible.  A kernel touches no global
+// memory before its pdl_wait (the previous kernel may still read or write it).  Both are no-ops
+// in a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void set_status(int32_t* dev_status, int32_t code) {
   if (dev_status) atomicCAS(dev_status, 0, code);
 }
 
 }  // namespace w4
+
+// Host: launch a kernel that may begin while the previous kernel on `stream` finishes
+// (programmatic stream serialization; the kernel synchronises with pdl_wait).
+template <typename... KArgs, typename... Args>
+static inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                     cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}

@@ -196,7 +196,9 @@ __global__ void __launch_bounds__(kFusedWarps * 32) route_fused_kernel(RouteArgs
   int* s_ids = s_off + A.E;                               // [T][k]
   int* s_wsum = s_ids + A.T * A.k;                        // [32]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_trigger();
   for (int i = threadIdx.x; i < A.E * W; i += blockDim.x) s_mask[i] = 0u;
+  pdl_wait();
   __syncthreads();
   topk_dispatch(A, 0, A.T, [&](int t, int e, int gl) {
     s_ids[t * A.k + gl] = e;
@@ -250,7 +252,9 @@ __global__ void __launch_bounds__(kFusedWarps * 32) route_fused_kernel(RouteArgs
 __global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(RouteArgs A) {
   extern __shared__ int smem[];
   int* s_cnt = smem;
+  pdl_trigger();
   for (int e = threadIdx.x; e < A.E; e += blockDim.x) s_cnt[e] = 0;
+  pdl_wait();
   __syncthreads();
   const int t0 = blockIdx.x * A.tokens_per_cta;
   const int t1 = min(A.T, t0 + A.tokens_per_cta);
@@ -265,6 +269,8 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_scatter_kernel(RouteAr
   int* s_base = s_tot + A.E;             // [E]
   int* s_wcnt = s_base + A.E;            // [nwarps][E]
   const int nctas = gridDim.x;
+  pdl_trigger();
+  pdl_wait();
   for (int e = threadIdx.x; e < A.E; e += blockDim.x) {
     int tot = 0, mine = 0;
     for (int c = 0; c < nctas; ++c) {
@@ -308,6 +314,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const uint16_t* __restrict
                                                       int T, int k, int H, uint16_t* __restrict__ y) {
   const int t = blockIdx.x;
   const int h8 = blockIdx.y * blockDim.x + threadIdx.x;
+  pdl_trigger();
+  pdl_wait();
   if (t >= T || h8 * 8 >= H) return;
   const int64_t T_k = static_cast<int64_t>(T) * k;
   int64_t row[KMAX];
@@ -386,16 +394,18 @@ w4_status w4_launch_route(const float* logits, int T, int E, int k, int32_t* ids
     // masks [E][ceil(T/32)], offsets [E], ids [T][k], warp sums [32]: <= 36 KB (E <= 1024)
     const size_t smem = (static_cast<size_t>(E) * ((T + 31) / 32) + E + static_cast<size_t>(T) * k + 32) *
                         sizeof(int);
-    w4::route_fused_kernel<<<1, w4::kFusedWarps * 32, smem, stream>>>(A);
+    if (launch_pdl(w4::route_fused_kernel, dim3(1), dim3(w4::kFusedWarps * 32), smem, stream, A) != cudaSuccess)
+      return W4_ERR_CUDA;
   } else {
     if (ws == nullptr || ws_bytes < w4_route_workspace_bytes(T, E)) return W4_ERR_WORKSPACE;
     A.hist = static_cast<int32_t*>(ws);
     A.scatter_warps = scatter_warps_for(E, w4::kRouteWarps);
     const size_t smem = static_cast<size_t>(2 + A.scatter_warps) * E * sizeof(int);
     const int nctas = route_num_ctas(T);
-    w4::route_topk_kernel<<<nctas, threads, E * sizeof(int), stream>>>(A);
-    if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
-    w4::route_scatter_kernel<<<nctas, threads, smem, stream>>>(A);
+    if (launch_pdl(w4::route_topk_kernel, dim3(nctas), dim3(threads), E * sizeof(int), stream, A) != cudaSuccess)
+      return W4_ERR_CUDA;
+    if (launch_pdl(w4::route_scatter_kernel, dim3(nctas), dim3(threads), smem, stream, A) != cudaSuccess)
+      return W4_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
@@ -405,7 +415,9 @@ w4_status w4_launch_combine(const uint16_t* o, const float* topk_w, const int32_
   if (T == 0) return W4_OK;
   const int threads = 128;
   dim3 grid(T, (H / 8 + threads - 1) / threads);
-  if (k <= 8) w4::combine_kernel<8><<<grid, threads, 0, stream>>>(o, topk_w, pair_pos, T, k, H, y);
-  else w4::combine_kernel<32><<<grid, threads, 0, stream>>>(o, topk_w, pair_pos, T, k, H, y);
+  cudaError_t e;
+  if (k <= 8) e = launch_pdl(w4::combine_kernel<8>, grid, dim3(threads), 0, stream, o, topk_w, pair_pos, T, k, H, y);
+  else e = launch_pdl(w4::combine_kernel<32>, grid, dim3(threads), 0, stream, o, topk_w, pair_pos, T, k, H, y);
+  if (e != cudaSuccess) return W4_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }

@@ -223,10 +223,13 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
   int* offs = table + (A.E + 1);
 
   // Activation and quad stages start zeroed: token columns past a block's rows then read finite
-  // values (their results are dropped).  The activation and quad areas are contiguous.
+  // values (their results are dropped).  The activation and quad areas are contiguous.  This
+  // set-up overlaps the end of the previous kernel on the stream; global memory waits for it.
+  // (No early trigger here: kernels after the GEMM launch when it completes.)
   for (int p = 0; p < kPipes; ++p)
     for (int i = threadIdx.x; i < S * (L.x_bytes + L.q_bytes) / 16; i += blockDim.x)
       reinterpret_cast<uint4*>(smem0 + p * L.pipe_bytes + L.x_off)[i] = make_uint4(0, 0, 0, 0);
+  pdl_wait();
 
   // unit table: table[e] = first unit of expert e, table[E] = total; offsets copied to offs[].
   // Offsets that are not non-decreasing from 0 to rows make the launch a no-op (W4_ERR_INVALID_ARG).
@@ -640,6 +643,8 @@ stream_prep_kernel(const uint16_t* __restrict__ a, const int32_t* __restrict__ a
   const int64_t wpb = blockDim.x >> 5;
   const int nv = K >> 3;                          // 8-element chunks in the row
   const int nblk = (K + kGS * 32 - 1) / (kGS * 32);
+  pdl_trigger();
+  pdl_wait();
   for (int64_t r = blockIdx.x * wpb + (threadIdx.x >> 5); r < rows; r += gridDim.x * wpb) {
     int64_t src = r;
     if (a_row_of_pair) {
@@ -870,8 +875,8 @@ static w4_status launch_one(const CUtensorMap& tmap, const CUtensorMap& smap, co
       return W4_ERR_CUDA;
     attr_done[dev] = 1;
   }
-  w4::stream_gemm_kernel<MT, GELU, SCALE><<<sm_count, w4::kThreads, A.L.total, stream>>>(tmap, smap, A);
-  return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+  return launch_pdl(w4::stream_gemm_kernel<MT, GELU, SCALE>, dim3(sm_count), dim3(w4::kThreads),
+                    A.L.total, stream, tmap, smap, A) == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
 template <int MT, bool GELU>
@@ -929,9 +934,9 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
     const int64_t a_rows = a_row_of_pair ? rows / kd : rows;
     const int64_t blocks = (rows + 7) / 8;
     const int grid = static_cast<int>(blocks < 16LL * sm_count ? blocks : 16LL * sm_count);
-    w4::stream_prep_kernel<<<grid, 256, 0, stream>>>(a, a_row_of_pair, kd, a_rows, rows, K, wsb,
-                                                     A.xw_stride, dev_status);
-    if (cudaGetLastError() != cudaSuccess) return W4_ERR_CUDA;
+    if (launch_pdl(w4::stream_prep_kernel, dim3(grid), dim3(256), 0, stream, a, a_row_of_pair, kd, a_rows,
+                   rows, K, wsb, A.xw_stride, dev_status) != cudaSuccess)
+      return W4_ERR_CUDA;
   }
   CUtensorMap tmap, smap;
   std::memset(&smap, 0, sizeof(smap));
