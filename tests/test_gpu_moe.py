@@ -11,7 +11,7 @@ import pytest
 import torch
 
 from oracle import bf16, moe
-from w4a16_group_quantized_w4_b200 import api, synth
+from w4a16_group_quantized_w4_b200 import _lib, api, synth
 from tests._util import assert_rows_close, dev_bf16, dev_f32, dev_u32, host_f64
 
 pytestmark = pytest.mark.gpu
@@ -123,6 +123,25 @@ def test_moe_decode_layer_full_config():
     case = synth.case_moe_decode()
     layer, y, ref = _layer(case)
     assert np.array_equal(layer.rt.sorted_pair.cpu().numpy(), ref.routing.sorted_pair)
+    assert_rows_close(host_f64(layer.h), ref.h, what="h")
+    assert_rows_close(host_f64(y), ref.y, what="y")
+
+
+@pytest.mark.parametrize("T", [1, 2, 3])
+def test_moe_small_batch_split_k(T):
+    """A few decode tokens through the full-size layer.  One token's 8 routed rows give the
+    gate/up GEMM only 88 units, so it splits K in three (the workspace then holds the float32
+    partials) and the last split of each tile reduces them and applies the GELU gate; 16 and 24
+    rows already fill more than half of the pipelines and take the unsplit path."""
+    case = synth.moe_case(T, 128, 8, 2816, 704, seed=90 + T)
+    rows = T * 8
+    prepared = 656 * (2816 // 256) * rows
+    ws = api.w4_workspace_bytes(_lib.W4_OP_GMM, rows, 2 * 704, 2816, 128, 8)
+    if T == 1:
+        assert ws > prepared + 3 * 4 * rows * 1408
+    else:
+        assert ws <= prepared + 256
+    layer, y, ref = _layer(case)
     assert_rows_close(host_f64(layer.h), ref.h, what="h")
     assert_rows_close(host_f64(y), ref.y, what="y")
 

@@ -38,8 +38,10 @@
 //     stage (a global load there would wait behind the weight stream).
 //   * Epilogue from registers, without a CTA barrier: with the GELU gate each warp's two A-fragment
 //     row sets are 8 gate rows and the 8 up rows of the same outputs, so h = gelu(g) * u is formed
-//     in the thread that holds both.  Dense split-K writes float32 partials that the last CTA of
-//     the tile reduces in a fixed order (deterministic).
+//     in the thread that holds both.  When the units would not cover the pipelines (dense GEMVs,
+//     grouped calls with a few routed rows, e.g. one decode token through 8 experts), K is split:
+//     float32 partials that the last pipeline of the tile reduces in a fixed order
+//     (deterministic), applying the GELU gate after the sum.
 // Rounding: the products are exact; each MMA sums 16 products of up to (1024 + 240) * 2^15 in
 // float32 next to the bias, which the correction cancels, so a group's sum carries an absolute
 // error of a few float32 units of its bias term (about 2^-13 of the group's mean |x'| times the
@@ -76,7 +78,7 @@ constexpr int kQPitch = kQBlock + 16;         // bytes per row pair in a stage's
 constexpr int kCodeBytes = kBN * kGS * 16;    // 16 KB
 constexpr int kBlockMaxKg = 24;               // scale-block mode: two 64-row blocks of <= 24 groups
 constexpr int kEpPitch = kBN + 4;             // floats per token row in the epilogue buffer
-constexpr int kDescBytes = 16;                // stage descriptor
+constexpr int kDescBytes = 32;                // stage descriptor
 constexpr int kPB = 12;                       // preparation pass: 256-k blocks per register batch
 // dynamic shared memory of the CTA (227 KB opt-in limit per block)
 constexpr int kSmemPerCta = 232448;
@@ -120,23 +122,26 @@ struct Unit {
   int64_t r0;
   int mt;
   int g0, g1;
+  int tile;               // dense id of (e, tb, nt)
 };
 
 // Stage descriptor written by the producer next to the stage's data, read by the compute warps
 // after the stage's full barrier: the unit the stage belongs to and where it sits in it.
 enum : int { kDescFirst = 1, kDescLast = 2, kDescDone = 4 };
-// One 16-byte load: {r0, first group, tile, mt | groups << 5 | flags << 9 | x << 12} where x is
-// the expert (no split-K) or the K split (split-K runs on one expert).
+// {r0, first group, weight tile, mt | groups << 5 | flags << 9} in the first 16 bytes (read every
+// stage), {expert, K split, tile id, 0} in the second (read only by the split-K epilogue and the
+// direct-load scale mode).  The tile id numbers the (expert, token block, weight tile) triples
+// 0.. densely; the split-K arrival counters are indexed by it.
 struct __align__(16) StageDesc {
   int r0;
   int g;
   int nt;
   int bits;
+  int e, sp, tile, pad;
 };
 __device__ __forceinline__ int desc_mt(const StageDesc& d) { return d.bits & 31; }
 __device__ __forceinline__ int desc_gc(const StageDesc& d) { return (d.bits >> 5) & 15; }
 __device__ __forceinline__ int desc_flags(const StageDesc& d) { return (d.bits >> 9) & 7; }
-__device__ __forceinline__ int desc_x(const StageDesc& d) { return d.bits >> 12; }
 
 // Unit u -> (expert, token block, tile, split); `table` and `offs` live in shared memory.
 template <int MT>
@@ -158,6 +163,7 @@ __device__ __forceinline__ void decode_unit(const StreamArgs& A, const int* tabl
   else { U.nt = rest / A.splits; U.sp = rest - U.nt * A.splits; }
   U.r0 = off0 + U.tb * MT;
   U.mt = min(MT, off1 - static_cast<int>(U.r0));
+  U.tile = table[U.e] / A.splits + U.tb + ntb * U.nt;
   U.g0 = U.sp * A.stages_per_split * kGS;
   U.g1 = min(A.kg, U.g0 + A.stages_per_split * kGS);
 }
@@ -316,7 +322,11 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           dsc.g = g;
           dsc.nt = U.nt;
           const int fl = (g == U.g0 ? kDescFirst : 0) | (g + kGS >= U.g1 ? kDescLast : 0);
-          dsc.bits = U.mt | (min(kGS, U.g1 - g) << 5) | (fl << 9) | ((A.splits > 1 ? U.sp : U.e) << 12);
+          dsc.bits = U.mt | (min(kGS, U.g1 - g) << 5) | (fl << 9);
+          dsc.e = U.e;
+          dsc.sp = U.sp;
+          dsc.tile = U.tile;
+          dsc.pad = 0;
           desc[slot] = dsc;
           uint32_t sbytes = 0;
           if (SCALE == kScaleTma) sbytes = 2 * kHalf * kGS * 2;
@@ -376,7 +386,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
   auto epi_sync = [&]() -> bool {
     __syncwarp();
     if (lane == 0) mbar_arrive(epi_bar);
-    const bool ok = mbar_wait(epi_bar, ephase);
+    const bool ok = mbar_wait_ring(epi_bar, ephase);
     ephase ^= 1u;
     if (!ok && lane == 0) { set_status(A.dev_status, W4_ERR_TIMEOUT); flags[0] = 1; }
     return ok;
@@ -395,7 +405,9 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       if (lane == 0) { set_status(A.dev_status, W4_ERR_TIMEOUT); flags[0] = 1; }
       return;
     }
-    const StageDesc dsc = desc[slot];
+    const int4 d0 = *reinterpret_cast<const int4*>(desc + slot);   // first half of the descriptor
+    StageDesc dsc;
+    dsc.r0 = d0.x; dsc.g = d0.y; dsc.nt = d0.z; dsc.bits = d0.w;
     const int dflags = desc_flags(dsc);
     if (dflags & kDescDone) return;
     const int g = dsc.g;
@@ -421,7 +433,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         shi[p] = 2 * p < gc ? phi[p] : 0u;
       }
     } else {
-      const int dnt = dsc.nt, de = A.splits > 1 ? 0 : desc_x(dsc);
+      const int dnt = dsc.nt, de = desc[slot].e;
       const int64_t grow_lo = tile_row_valid(A, dnt, rlo) ? tile_row(A, de, dnt, rlo) : tile_row(A, de, dnt, 0);
       const int64_t grow_hi = tile_row_valid(A, dnt, rhi) ? tile_row(A, de, dnt, rhi) : tile_row(A, de, dnt, 0);
 #pragma unroll
@@ -519,7 +531,13 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       }
     }
     const bool last = dflags & kDescLast;
+    int sp_last = 0, tile_last = 0;     // the unit's K split and tile id (split-K epilogue)
     if (last) {
+      if (A.splits > 1) {
+        const int4 d1 = reinterpret_cast<const int4*>(desc + slot)[1];   // before the slot is freed
+        sp_last = d1.y;
+        tile_last = d1.z;
+      }
       // undo the activation rows' power-of-two exponents (token columns 2tq, 2tq + 1 of each
       // block; the multipliers travel with the rows, so no global load waits behind the stream)
 #pragma unroll
@@ -565,8 +583,8 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         }
       }
     } else {
-      // split-K (dense, no gate): float32 partials through shared memory, then the last CTA of
-      // the tile reduces them in split order
+      // split-K: float32 partials through shared memory, then the last pipeline to finish its
+      // part of the tile reduces them in split order (and applies the GELU gate)
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
         const int t0 = b * 8 + 2 * tq;
@@ -577,12 +595,25 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       }
       if (!epi_sync()) return;
       const int ctid = warp * 32 + lane;
-      const int n0 = nt * kBN;
+      const int Nh = A.N >> 1;
+      // partial column of tile row c (GELU: rows 0..63 gate j, 64..127 up j of outputs j)
+      auto pcol = [&](int c, bool& ok) -> int {
+        if (gelu) {
+          const int j = nt * kHalf + (c & (kHalf - 1));
+          ok = j < Nh;
+          return c < kHalf ? j : Nh + j;
+        }
+        const int n = nt * kBN + c;
+        ok = n < A.N;
+        return n;
+      };
       if (!flags[0]) {
         for (int idx = ctid; idx < mt * kBN; idx += kWarps * 32) {
           const int t = idx / kBN, c = idx % kBN;
-          if (n0 + c < A.N)
-            A.partial[(static_cast<int64_t>(desc_x(dsc)) * A.rows + r0 + t) * A.N + n0 + c] = ep[t * kEpPitch + c];
+          bool ok;
+          const int n = pcol(c, ok);
+          if (ok)
+            A.partial[(static_cast<int64_t>(sp_last) * A.rows + r0 + t) * A.N + n] = ep[t * kEpPitch + c];
         }
       }
       __threadfence();
@@ -590,31 +621,41 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       if (ctid == 0) {
         int last = 0;
         if (!flags[0]) {
-          const int tile = ((dsc.r0 - offs[0]) / MT) * A.n_tiles + nt;   // dense: one expert
-          const int prev = atomicAdd(&A.counters[tile], 1);
+          const int prev = atomicAdd(&A.counters[tile_last], 1);
           last = (prev == A.splits - 1);
-          if (last) A.counters[tile] = 0;
+          if (last) A.counters[tile_last] = 0;
         }
         flags[1] = last;
       }
       if (!epi_sync()) return;
       if (flags[1]) {
         __threadfence();
-        for (int idx = ctid; idx < mt * kBN; idx += kWarps * 32) {
-          const int t = idx / kBN, c = idx % kBN;
-          if (n0 + c < A.N) {
-            // the partials of up to 8 splits are loaded together, then summed in split order
-            const float* pp = A.partial + (r0 + t) * A.N + n0 + c;
-            const int64_t ps = A.rows * A.N;
-            float sum = 0.f;
-            for (int sp0 = 0; sp0 < A.splits; sp0 += 8) {
-              float pv[8];
+        const int64_t ps = A.rows * A.N;
+        // the partials of up to 8 splits are loaded together, then summed in split order
+        auto sum_col = [&](int t, int n) -> float {
+          const float* pp = A.partial + (r0 + t) * A.N + n;
+          float sum = 0.f;
+          for (int sp0 = 0; sp0 < A.splits; sp0 += 8) {
+            float pv[8];
 #pragma unroll
-              for (int q = 0; q < 8; ++q) pv[q] = sp0 + q < A.splits ? __ldcg(pp + (sp0 + q) * ps) : 0.f;
+            for (int q = 0; q < 8; ++q) pv[q] = sp0 + q < A.splits ? __ldcg(pp + (sp0 + q) * ps) : 0.f;
 #pragma unroll
-              for (int q = 0; q < 8; ++q) sum += pv[q];
-            }
-            A.out[(r0 + t) * A.N + n0 + c] = f32_to_bf16_bits(sum);
+            for (int q = 0; q < 8; ++q) sum += pv[q];
+          }
+          return sum;
+        };
+        if (gelu) {
+          for (int idx = ctid; idx < mt * kHalf; idx += kWarps * 32) {
+            const int t = idx / kHalf, c = idx % kHalf;
+            const int j = nt * kHalf + c;
+            if (j < Nh)
+              A.out[(r0 + t) * Nh + j] = f32_to_bf16_bits(gelu_tanh(sum_col(t, j)) * sum_col(t, Nh + j));
+          }
+        } else {
+          const int n0 = nt * kBN;
+          for (int idx = ctid; idx < mt * kBN; idx += kWarps * 32) {
+            const int t = idx / kBN, c = idx % kBN;
+            if (n0 + c < A.N) A.out[(r0 + t) * A.N + n0 + c] = f32_to_bf16_bits(sum_col(t, n0 + c));
           }
         }
       }
@@ -822,16 +863,20 @@ static StreamPlan plan_stream(int64_t rows, int N, int K, int E, int epi, bool d
   p.n_tiles = (epi == W4_EPI_GELU_GATE) ? ((N / 2) + w4::kHalf - 1) / w4::kHalf
                                         : (N + w4::kBN - 1) / w4::kBN;
   p.splits = 1;
-  if (dense) {
-    // split K only while the units cover fewer than ~3/4 of the pipelines (long units stream
-    // better than many short ones: a K = 4096 GEMV measured fastest with two splits) and the
-    // float32 partials stay below ~1/8 of the weight bytes
-    const int64_t ntb = (rows + p.MT - 1) / p.MT;
-    const double wbytes = static_cast<double>(N) * K * 0.5625;
-    while (p.splits * 2 <= kstages && 4 * ntb * p.n_tiles * p.splits < 3LL * w4::kPipes * sm_count &&
-           static_cast<double>(p.splits * 2) * rows * N * 8.0 <= wbytes / 8.0)
-      p.splits *= 2;
-  }
+  // Split K into as many parts as keep all units within one wave of the pipelines (long units
+  // stream better than many short ones: a K = 4096 GEMV measured fastest with two splits, and a
+  // second wave of split units costs more than it saves), with at least two stages per part and
+  // float32 partials below ~1/8 of the weight bytes.  Grouped calls count the token blocks the
+  // most spread-out routing can produce: at most one per row, and at most one per expert plus
+  // one per MT rows.
+  const int64_t ntb = dense ? (rows + p.MT - 1) / p.MT
+                            : std::min<int64_t>(rows, static_cast<int64_t>(E) + rows / p.MT);
+  const int64_t units = std::max<int64_t>(1, ntb * p.n_tiles);
+  const double wbytes = static_cast<double>(E) * N * K * 0.5625;
+  int64_t sp = static_cast<int64_t>(w4::kPipes) * sm_count / units;
+  sp = std::min<int64_t>(sp, kstages / 2);
+  while (sp > 1 && static_cast<double>(sp) * rows * N * 4.0 > wbytes / 8.0) --sp;
+  p.splits = sp > 1 ? static_cast<int>(sp) : 1;
   p.stages_per_split = (kstages + p.splits - 1) / p.splits;
   p.splits = (kstages + p.stages_per_split - 1) / p.stages_per_split;
   return p;
@@ -850,8 +895,10 @@ static size_t prep_bytes(int64_t rows, int K) {
   return align256(static_cast<size_t>(rows) * prep_stride(K));
 }
 
-static size_t counters_bytes(const StreamPlan& p, int64_t rows) {
-  const int64_t ntb = (rows + p.MT - 1) / p.MT;
+// one arrival counter per (expert, token block, weight tile): at most min(E, rows) + rows / MT
+// token blocks over all experts
+static size_t counters_bytes(const StreamPlan& p, int64_t rows, int E) {
+  const int64_t ntb = std::min<int64_t>(E, rows) + (rows + p.MT - 1) / p.MT;
   return align256(static_cast<size_t>(ntb * p.n_tiles) * sizeof(int32_t));
 }
 
@@ -859,7 +906,7 @@ size_t w4_stream_workspace_bytes(int64_t rows, int N, int K, int E, int epi, boo
   if (rows <= 0) return 0;
   StreamPlan p = plan_stream(rows, N, K, E, epi, dense, sm_count);
   size_t b = prep_bytes(rows, K);
-  if (p.splits > 1) b += counters_bytes(p, rows) + static_cast<size_t>(p.splits) * rows * N * sizeof(float);
+  if (p.splits > 1) b += counters_bytes(p, rows, E) + static_cast<size_t>(p.splits) * rows * N * sizeof(float);
   return b;
 }
 
@@ -906,7 +953,7 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
   int scale_mode;
   if (A.kg % 8 == 0 && s16) {
     scale_mode = w4::kScaleTma;
-  } else if (p.splits == 1 && A.kg % 2 == 0 && A.kg <= w4::kBlockMaxKg && N % 8 == 0 && s16 &&
+  } else if (A.kg % 2 == 0 && A.kg <= w4::kBlockMaxKg && N % 8 == 0 && s16 &&
              (epi == W4_EPI_GELU_GATE ? (N / 2) % w4::kHalf == 0 : N % w4::kBN == 0)) {
     // (whole tiles only: the 64-row blocks are plain bulk copies and must stay inside the array)
     scale_mode = w4::kScaleBlock;
@@ -923,7 +970,7 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
   A.xw_stride = prep_stride(K);
   if (p.splits > 1) {
     uint8_t* cbase = wsb + prep_bytes(rows, K);
-    const size_t cb = counters_bytes(p, rows);
+    const size_t cb = counters_bytes(p, rows, E);
     A.counters = reinterpret_cast<int32_t*>(cbase);
     A.partial = reinterpret_cast<float*>(cbase + cb);
     // the arrival counters must start at zero whatever the workspace held before
