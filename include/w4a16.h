@@ -197,7 +197,7 @@ w4_status moe_combine(const uint16_t* o, const float* topk_w, const int32_t* pai
  *     row's scratch exceeds 8 MiB (8388608 bytes).
  *   - The first call on a device looks up the array's device address (once per device); make
  *     that first call before any stream capture.
- *   - Every call reuses the same array (clearing its arrival counters with a cudaMemsetAsync on
+ *   - Every call reuses the same array (its kernels clear the arrival counters they use, on
  *     `stream`): calls that overlap on the GPU race and must be ordered by the caller (one
  *     stream, or events).
  *   - Allocates nothing: no cudaMalloc/cudaFree, no allocating library routine.

@@ -679,13 +679,16 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
 __global__ void __launch_bounds__(256)
 stream_prep_kernel(const uint16_t* __restrict__ a, const int32_t* __restrict__ a_row_of_pair, int k_div,
                    int64_t a_rows, int64_t rows, int K, uint8_t* __restrict__ xw, int64_t stride,
-                   int32_t* dev_status) {
+                   int32_t* __restrict__ counters, int n_counters, int32_t* dev_status) {
   const int lane = threadIdx.x & 31;
   const int64_t wpb = blockDim.x >> 5;
   const int nv = K >> 3;                          // 8-element chunks in the row
   const int nblk = (K + kGS * 32 - 1) / (kGS * 32);
   pdl_trigger();
   pdl_wait();
+  // the GEMM's split-K arrival counters start at zero whatever the workspace held before
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_counters; i += gridDim.x * blockDim.x)
+    counters[i] = 0;
   for (int64_t r = blockIdx.x * wpb + (threadIdx.x >> 5); r < rows; r += gridDim.x * wpb) {
     int64_t src = r;
     if (a_row_of_pair) {
@@ -973,16 +976,16 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
     const size_t cb = counters_bytes(p, rows, E);
     A.counters = reinterpret_cast<int32_t*>(cbase);
     A.partial = reinterpret_cast<float*>(cbase + cb);
-    // the arrival counters must start at zero whatever the workspace held before
-    if (cudaMemsetAsync(cbase, 0, cb, stream) != cudaSuccess) return W4_ERR_CUDA;
+    // (the preparation pass clears the arrival counters)
   }
   {
     const int kd = k_div > 0 ? k_div : 1;
     const int64_t a_rows = a_row_of_pair ? rows / kd : rows;
     const int64_t blocks = (rows + 7) / 8;
     const int grid = static_cast<int>(blocks < 16LL * sm_count ? blocks : 16LL * sm_count);
+    const int n_counters = p.splits > 1 ? static_cast<int>(counters_bytes(p, rows, E) / sizeof(int32_t)) : 0;
     if (launch_pdl(w4::stream_prep_kernel, dim3(grid), dim3(256), 0, stream, a, a_row_of_pair, kd, a_rows,
-                   rows, K, wsb, A.xw_stride, dev_status) != cudaSuccess)
+                   rows, K, wsb, A.xw_stride, A.counters, n_counters, dev_status) != cudaSuccess)
       return W4_ERR_CUDA;
   }
   CUtensorMap tmap, smap;
