@@ -128,6 +128,18 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
 
+// L2 prefetch of one 2-D tensor tile (no shared-memory destination, nothing to wait for).  The
+// innermost coordinate obeys the same 16-byte rule as a tile load.
+__device__ __forceinline__ void tma_prefetch_2d(const void* tmap, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+               ::"l"(tmap), "r"(x), "r"(y) : "memory");
+}
+
+// L2 prefetch of a contiguous range: src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ------------------------------------------------------------------------------------------
 // loads
 // ------------------------------------------------------------------------------------------
