@@ -23,7 +23,9 @@ namespace w4 {
 
 constexpr int kRouteWarps = 8;                 // warps per CTA in the two-launch path
 constexpr int kFusedWarps = 32;                // warps of the single-CTA path
-constexpr int kRouteTokensPerCta = 64;         // tokens per CTA in the two-launch path
+constexpr int kRouteTokensMin = 16;            // tokens per CTA in the two-launch path: from 16
+constexpr int kRouteTokensMax = 64;            // (top-k spread over many SMs) up to 64 (fewer
+                                               // histograms for the scatter to read)
 constexpr int kFusedMaxT = 128;                // largest T routed by the single-CTA path
 
 struct RouteArgs {
@@ -364,7 +366,12 @@ __global__ void __launch_bounds__(128) combine_kernel(const uint16_t* __restrict
 // host launchers (declared in api.cu)
 // ---------------------------------------------------------------------------------------------
 
-static int route_num_ctas(int T) { return (T + w4::kRouteTokensPerCta - 1) / w4::kRouteTokensPerCta; }
+// The top-k is ALU-bound per SM: spread the tokens over about 128 CTAs, 16 to 64 tokens each.
+static int route_tokens_per_cta(int T) {
+  int t = (T + 127) / 128;
+  return t < w4::kRouteTokensMin ? w4::kRouteTokensMin : (t > w4::kRouteTokensMax ? w4::kRouteTokensMax : t);
+}
+static int route_num_ctas(int T) { return (T + route_tokens_per_cta(T) - 1) / route_tokens_per_cta(T); }
 
 size_t w4_route_workspace_bytes(int T, int E) {
   if (T <= w4::kFusedMaxT) return 0;   // fused single-CTA path
@@ -382,7 +389,7 @@ w4_status w4_launch_route(const float* logits, int T, int E, int k, int32_t* ids
                           int32_t* offsets, int32_t* sorted_pair, int32_t* pair_pos, void* ws,
                           size_t ws_bytes, cudaStream_t stream) {
   w4::RouteArgs A{logits, T, E, k, ids, w, offsets, sorted_pair, pair_pos, nullptr,
-                  w4::kRouteTokensPerCta, 1};
+                  route_tokens_per_cta(T), 1};
   const int threads = w4::kRouteWarps * 32;
   // (2 + warps) * E ints <= 40 KB for E <= 1024: within the default shared-memory limit
   if (T == 0) {
