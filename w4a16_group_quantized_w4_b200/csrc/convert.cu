@@ -34,32 +34,53 @@ a_to_f16_kernel(const uint16_t* __restrict__ a, const int32_t* __restrict__ a_ro
       }
     }
     const uint4* src = reinterpret_cast<const uint4*>(a + srow * K);
+    // lane l holds chunks l, l + 32, ... of up to kCB * 32 chunks at a time, all loads in
+    // flight together; a row of at most kCB * 256 elements (K <= 3072) is read once
+    constexpr int kCB = 12;
+    uint4 v[kCB];
     uint32_t m = 0;
-    for (int i = lane; i < nv; i += 32) {
-      const uint4 v = __ldg(src + i);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int i0 = 0; i0 < nv; i0 += 32 * kCB) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t lo = w[j] & 0x7FFFu, hi = (w[j] >> 16) & 0x7FFFu;
-        if (lo < 0x7F80u) m = max(m, lo);
-        if (hi < 0x7F80u) m = max(m, hi);
+      for (int t = 0; t < kCB; ++t) {
+        const int i = i0 + 32 * t + lane;
+        v[t] = i < nv ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int t = 0; t < kCB; ++t) {
+        const uint32_t w[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t lo = w[j] & 0x7FFFu, hi = (w[j] >> 16) & 0x7FFFu;
+          if (lo < 0x7F80u) m = max(m, lo);
+          if (hi < 0x7F80u) m = max(m, hi);
+        }
       }
     }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    m = __reduce_max_sync(0xffffffffu, m);
     const int f = shift_for(m, 14);
     const float mul = pow2f(f);
     uint4* dst = reinterpret_cast<uint4*>(a16 + row * K);
-    for (int i = lane; i < nv; i += 32) {
-      const uint4 v = __ldg(src + i);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-      uint32_t o[4];
+    for (int i0 = 0; i0 < nv; i0 += 32 * kCB) {
+      if (nv > 32 * kCB) {                       // long rows: the batch again (from L1 / L2)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const __half2 h = __floats2half2_rn(bf16_lo_to_f32(w[j]) * mul, bf16_hi_to_f32(w[j]) * mul);
-        o[j] = *reinterpret_cast<const uint32_t*>(&h);
+        for (int t = 0; t < kCB; ++t) {
+          const int i = i0 + 32 * t + lane;
+          v[t] = i < nv ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+        }
       }
-      dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+      for (int t = 0; t < kCB; ++t) {
+        const int i = i0 + 32 * t + lane;
+        if (i >= nv) break;
+        const uint32_t w[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __half2 h = __floats2half2_rn(bf16_lo_to_f32(w[j]) * mul, bf16_hi_to_f32(w[j]) * mul);
+          o[j] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
     }
     if (lane == 0) rowmul[row] = pow2f(-f);
   }

@@ -97,7 +97,7 @@ struct Args {
 // 128-row token tiles.
 template <int NMAX, int KSK, int TSTAGES, int ASLOTS, int NSPLIT, int KSPLIT, int ABUF, int EPIW>
 struct Cfg {
-  static_assert(NMAX % 16 == 0 && NMAX <= 256, "MMA N");
+  static_assert(NMAX % 32 == 0 && NMAX <= 256, "MMA N, whole 32-token epilogue groups");
   static_assert(KSK == 128 || KSK == 256, "stage width");
   static constexpr int kSubs = KSK / 64;                 // 64-k token sub-tiles per stage
   static constexpr int kHalves = KSK / 128;              // TMEM A slots per stage
@@ -418,6 +418,18 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       Tile T;
       decode_tile(A, table, offs, t, NMAX, T);
       const int ab = ti % ABUF, hb = ti & 1;
+      // the multipliers of the tile's tokens this warp finishes, loaded before the accumulator
+      // wait so that their latency overlaps the tile's MMAs: with one warp per quadrant, lane l of
+      // register m holds token 32m + l; with two, part cp finishes tokens 32j + 16cp + i (i < 16)
+      // and lane l of register m holds the one with j = 2m + l / 16, i = l % 16
+      constexpr int kRJ = NMAX / 32;
+      constexpr int kRR = EPIW == 2 ? (kRJ + 1) / 2 : kRJ;
+      float rmr[kRR];
+#pragma unroll
+      for (int m = 0; m < kRR; ++m) {
+        const int tk = EPIW == 2 ? 32 * (2 * m + (lane >> 4)) + 16 * cp + (lane & 15) : 32 * m + lane;
+        rmr[m] = tk < T.mrows ? __ldg(A.rowmul + T.r0 + tk) : 0.f;
+      }
       if (!mbar_wait(&acc_full[ab], (ti / ABUF) & 1)) { fail(lane); break; }
       tc_fence_after();
       if (!mbar_wait(&sh_full[hb], (ti >> 1) & 1)) { fail(lane); break; }
@@ -427,6 +439,13 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       const int n_cols = (T.mrows + 15) & ~15;
       for (int c0 = 16 * cp; c0 < n_cols; c0 += 16 * EPIW) {
+        // this chunk's multipliers: register c0 / 64 (two warps per quadrant) or c0 / 32 (one),
+        // lanes sl .. sl + 15, picked by selects so that the array stays in registers
+        const int m = EPIW == 2 ? c0 >> 6 : c0 >> 5;
+        float rj = rmr[0];
+#pragma unroll
+        for (int mm = 1; mm < kRR; ++mm) rj = mm == m ? rmr[mm] : rj;
+        const int sl = EPIW == 2 ? (c0 & 32) >> 1 : c0 & 16;
         float v[16];
         tmem_ld16(taddr + C::acc_col(ab, 0) + c0, v);
 #pragma unroll
@@ -436,21 +455,8 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] += w[i];
         }
-        // the 16 token rows' multipliers: four 16-byte loads when the chunk is whole and aligned
-        float rm[16];
-        const float* rp = A.rowmul + T.r0 + c0;
-        if (c0 + 16 <= T.mrows && (reinterpret_cast<uintptr_t>(rp) & 15) == 0) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float4 f = __ldg(reinterpret_cast<const float4*>(rp) + i);
-            rm[4 * i] = f.x; rm[4 * i + 1] = f.y; rm[4 * i + 2] = f.z; rm[4 * i + 3] = f.w;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) rm[i] = c0 + i < T.mrows ? __ldg(rp + i) : 0.f;
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = (v[i] * rm[i]) * cm;
+        for (int i = 0; i < 16; ++i) v[i] = (v[i] * __shfl_sync(0xffffffffu, rj, sl + i)) * cm;
         if (gelu) {
           // lanes i < 16: gate values, lanes i + 16: up values of the same output j; the lower
           // lane finishes tokens c0 .. c0+7, the upper one tokens c0+8 .. c0+15
@@ -727,8 +733,9 @@ w4_status w4_launch_tm_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int
   A.n_tiles = (epi == W4_EPI_GELU_GATE) ? (N / 2) / (w4::tm::kBM / 2) : N / w4::tm::kBM;
   A.dev_status = dev_status;
   const uint16_t* a16 = w4_ws_a16(ws);
-  // 192-row token blocks, 128-k stages with three token stages in flight, two MMA-issuing
-  // threads (96 token columns each: the tensor pipe's rate needs more than one issuer), two
-  // 192-column accumulators drained by eight epilogue warps
-  return tm_launch_cfg<192, 128, 3, 2, 2, 1, 2, 2>(codes, a16, rows, K, A, stream, sm_count);
+  // 192-row token blocks, 128-k stages with three token stages in flight, one MMA-issuing thread
+  // (N = 192: every tcgen05.mma costs a fixed time on top of its columns, so fewer, wider MMAs
+  // finish sooner than two threads' 96-column ones), two 192-column accumulators drained by eight
+  // epilogue warps
+  return tm_launch_cfg<192, 128, 3, 2, 1, 1, 2, 2>(codes, a16, rows, K, A, stream, sm_count);
 }
