@@ -70,6 +70,7 @@ constexpr int kACols = 64;                               // TMEM columns per A s
 struct Lay {
   int code;                 // code ring: cst stages
   int cst;
+  int stage;                // epilogue output staging: 2 x 1 KB per epilogue warp
   int sh;                   // float [2][128]: 2^-e per TMEM lane
   int bars;
   int tmem_slot;            // + abort flag
@@ -88,6 +89,7 @@ struct Args {
   uint16_t* out;
   int n_tiles;              // weight tiles per expert
   int32_t* dev_status;
+  int tma_out;              // 1: whole 16-token chunks leave through shared memory and TMA stores
   Lay L;
 };
 
@@ -209,7 +211,8 @@ __device__ __forceinline__ void scale_pair(uint32_t s16, float smul, uint32_t& s
 template <int NMAX, int KSK, int TSTAGES, int ASLOTS, int NSPLIT, int KSPLIT, int ABUF, int EPIW>
 __global__ void __launch_bounds__(32 * (16 + (NSPLIT * KSPLIT - 1) + 4 * (EPIW - 1)), 1)
 tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
-               const __grid_constant__ CUtensorMap tmap_tok, Args A) {
+               const __grid_constant__ CUtensorMap tmap_tok,
+               const __grid_constant__ CUtensorMap tmap_out, Args A) {
   using C = Cfg<NMAX, KSK, TSTAGES, ASLOTS, NSPLIT, KSPLIT, ABUF, EPIW>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -413,6 +416,12 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     const int cp = warp < 8 ? 0 : 1;
     const int l = q * 32 + lane;
     const bool gelu = A.epi == W4_EPI_GELU_GATE;
+    // A whole 16-token chunk is written to one of this warp's two 1 KB buffers as a [16 token]
+    // x [32 outputs] (GELU: [16] x [16]) bf16 box and leaves by one TMA store, so the stores do
+    // not hold the warp; a ragged chunk (the last of an expert's block) is stored element by
+    // element and never touches the next block's rows.
+    uint8_t* stg = smem + L.stage + (q + 4 * cp) * 2048;
+    int n_out = 0;                                 // TMA stores issued by this warp (lane 0)
     int ti = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++ti) {
       Tile T;
@@ -457,7 +466,35 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         }
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = (v[i] * __shfl_sync(0xffffffffu, rj, sl + i)) * cm;
-        if (gelu) {
+        if (A.tma_out && c0 + 16 <= T.mrows) {
+          uint16_t* buf = reinterpret_cast<uint16_t*>(stg + (n_out & 1) * 1024);
+          if (n_out >= 2) {                         // the store that last read this buffer
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+          }
+          if (gelu) {
+            const bool upper = lane >= 16;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float send = upper ? v[i] : v[8 + i];
+              const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+              const float g = upper ? recv : v[i];
+              const float u = upper ? v[8 + i] : recv;
+              buf[(i + (upper ? 8 : 0)) * 16 + (lane & 15)] = f32_to_bf16_bits(gelu_tanh(g) * u);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) buf[i * 32 + lane] = f32_to_bf16_bits(v[i]);
+          }
+          fence_proxy_async();                      // the generic writes, before the async read
+          __syncwarp();
+          if (lane == 0) {
+            const int x = gelu ? T.nt * (kBM / 2) + 16 * q : T.nt * kBM + 32 * q;
+            tma_store_2d(&tmap_out, x, static_cast<int32_t>(T.r0 + c0), buf);
+            bulk_commit();
+          }
+          ++n_out;
+        } else if (gelu) {
           // lanes i < 16: gate values, lanes i + 16: up values of the same output j; the lower
           // lane finishes tokens c0 .. c0+7, the upper one tokens c0+8 .. c0+15
           const bool upper = lane >= 16;
@@ -486,6 +523,8 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[ab]);
     }
+    if (lane == 0) bulk_wait_all();              // this warp's stores are complete before exit
+    __syncwarp();
   } else if (warp >= 8) {
     // ------------------------------ dequant ------------------------------
     // warp 8 + 4h + q: TMEM lanes 32q .. 32q+31 (one weight row each), and in every 128-k slot the
@@ -646,12 +685,14 @@ static bool tm_layout(int E, int kg, w4::tm::Lay& L) {
   using C = w4::tm::Cfg<NMAX, KSK, TSTAGES, ASLOTS, NSPLIT, KSPLIT, ABUF, EPIW>;
   (void)kg;
   L.code = C::code;
-  const int fixed = 2 * w4::tm::kBM * 4 + C::nbars * 8 + 16 + (E + 1) * 8;
+  const int stage = C::kEpiWarps * 2048;
+  const int fixed = stage + 2 * w4::tm::kBM * 4 + C::nbars * 8 + 16 + (E + 1) * 8;
   int cst = (kTmSmemBudget - L.code - fixed) / C::kCodeStage;
   if (cst > w4::tm::kMaxCStages) cst = w4::tm::kMaxCStages;
   if (cst < 2) return false;
   L.cst = cst;
-  L.sh = L.code + cst * C::kCodeStage;
+  L.stage = L.code + cst * C::kCodeStage;     // 1024-byte aligned (whole code stages)
+  L.sh = L.stage + stage;
   L.bars = L.sh + 2 * w4::tm::kBM * 4;
   L.tmem_slot = L.bars + C::nbars * 8;
   L.table = L.tmem_slot + 16;
@@ -692,6 +733,25 @@ static w4_status tm_launch_cfg(const uint32_t* codes, const uint16_t* a16, int64
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return W4_ERR_CUDA;
   }
+  // routed outputs [rows, N] (GELU: [rows, N / 2]) bf16: box = 32 (GELU: 16) outputs x 16 rows,
+  // unswizzled, for the epilogue's whole-chunk stores; without a usable map every element is
+  // stored directly
+  CUtensorMap tmap_out;
+  std::memset(&tmap_out, 0, sizeof(tmap_out));
+  A.tma_out = 0;
+  {
+    const bool gelu = A.epi == W4_EPI_GELU_GATE;
+    const int64_t nout = gelu ? A.N / 2 : A.N;
+    if ((reinterpret_cast<uintptr_t>(A.out) & 15) == 0 && (nout * 2) % 16 == 0 && rows >= 16) {
+      cuuint64_t dims[2] = {static_cast<cuuint64_t>(nout), static_cast<cuuint64_t>(rows)};
+      cuuint64_t strides[1] = {static_cast<cuuint64_t>(nout) * 2};
+      cuuint32_t box[2] = {gelu ? 16u : 32u, 16u};
+      if (fn(&tmap_out, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, A.out, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+        A.tma_out = 1;
+    }
+  }
   const size_t smem = static_cast<size_t>(A.L.total) + 1024;
   static int attr_done[64] = {0};
   int dev = 0;
@@ -703,7 +763,7 @@ static w4_status tm_launch_cfg(const uint32_t* codes, const uint16_t* a16, int64
     attr_done[dev] = 1;
   }
   w4::tm::tm_gemm_kernel<NMAX, KSK, TSTAGES, ASLOTS, NSPLIT, KSPLIT, ABUF, EPIW>
-      <<<sm_count, 32 * C::kWarps, smem, stream>>>(tmap_codes, tmap_tok, A);
+      <<<sm_count, 32 * C::kWarps, smem, stream>>>(tmap_codes, tmap_tok, tmap_out, A);
   return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
