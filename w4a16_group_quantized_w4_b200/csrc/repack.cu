@@ -6,7 +6,7 @@
 // The exact rule (float64, tolerance 1/16, off-grid fallback, zero and non-finite groups) is the
 // one stated beside w4_repack in w4a16.h; results are bit-identical to it.
 //
-// Work mapping: four lanes per group (64 input bytes -> 16 code bytes, 2 scale bytes, 1 m byte),
+// Work mapping: one lane per group (64 input bytes -> 16 code bytes, 2 scale bytes, 1 m byte),
 // grid-stride over all groups.  HBM-bound when the ALU work per group stays small, so the
 // m-search runs in float32 with a guard band and only falls back to the exact float64 search
 // when the float32 evidence cannot decide:
@@ -87,33 +87,20 @@ __device__ __noinline__ int search_exact(const GroupBits& g, double a, uint32_t 
   return 0;
 }
 
-// Work mapping: four consecutive lanes (a quad) per group; lane `sub` of the quad holds elements
-// 8 sub .. 8 sub + 7 (one 16-byte load) and produces code word `sub`.  Decisions that involve the
-// whole group (largest magnitude, pass / fail of a step, the least-squares sums) combine the four
-// lanes with shuffles inside the quad.
-__device__ __forceinline__ uint32_t quad_max(uint32_t v, unsigned qm) {
-  v = max(v, __shfl_xor_sync(qm, v, 1));
-  return max(v, __shfl_xor_sync(qm, v, 2));
-}
-__device__ __forceinline__ uint32_t quad_min(uint32_t v, unsigned qm) {
-  v = min(v, __shfl_xor_sync(qm, v, 1));
-  return min(v, __shfl_xor_sync(qm, v, 2));
-}
-__device__ __forceinline__ uint32_t quad_or(uint32_t v, unsigned qm) {
-  v |= __shfl_xor_sync(qm, v, 1);
-  return v | __shfl_xor_sync(qm, v, 2);
-}
-
-// float32 guard-band search over this lane's 8 elements (v: element 2j in the low half of v[j]),
-// decided for the quad.  Returns m in 1..8 (this lane's code word in cw), or 0 when the exact
-// path must decide.  An m for which the smallest nonzero |w| maps to r strictly inside
-// (1/16, 15/16) cannot reproduce the group (that element is more than 1/16 from every integer),
-// so it is skipped without looking at the elements (margins of 2^-16 cover the float32 error of
+// Work mapping: one lane per group.  The lane holds the group's 64 input bytes (four 16-byte
+// loads issued together, and the next group's four issued before this one is decided), so a
+// warp decides 32 groups at once and the per-group tail (float64 sum, division, bf16 rounding)
+// is shared by 32 groups per warp instruction.
+//
+// float32 guard-band search over the group (v: element 2j in the low half of v[j]).  Returns m
+// in 1..8 (code words in cw, least-squares sums in num / den), or 0 when the exact path must
+// decide.  An m for which the smallest nonzero |w| maps to r strictly inside (1/16, 15/16)
+// cannot reproduce the group (that element is more than 1/16 from every integer), so it is
+// skipped without looking at the elements (margins of 2^-16 cover the float32 error of
 // m * wmin / a); on the grid this makes the group's own m the first candidate.  The search runs
-// in rounds over the whole warp: each round every undecided group tries its next candidate, so
-// the eight groups of a warp share one pass instead of one pass per distinct m.
-__device__ __forceinline__ int search_fast_quad(const uint32_t (&v)[4], float a, float wmin,
-                                                unsigned qm, uint32_t& cw, float& psum, float& qsum) {
+// in rounds over the whole warp: each round every undecided group tries its next candidate.
+__device__ __forceinline__ int search_fast(const uint32_t (&v)[16], float a, float wmin,
+                                           uint32_t (&cw)[4], double& num, int& den) {
   const float tol = 0.0625f, band = 0x1p-17f, kRound = 12582912.0f;
   const float ra = __frcp_rn(a);
   const float rmin1 = __fmul_rn(wmin, ra);
@@ -128,11 +115,13 @@ __device__ __forceinline__ int search_fast_quad(const uint32_t (&v)[4], float a,
   const unsigned active = __activemask();
   while (__any_sync(active, !done)) {
     const float inv = __fmul_rn(static_cast<float>(next <= 8 ? next : 8), ra);
-    uint32_t t = 0, ubits = 0;
-    float dmax = 0.f, ps = 0.f, qs = 0.f;
+    uint32_t t[4] = {0u, 0u, 0u, 0u}, ubits = 0;
+    float dmax = 0.f, qs = 0.f;
+    float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float x = (i & 1) ? __uint_as_float(v[i >> 1] & 0xFFFF0000u) : __uint_as_float(v[i >> 1] << 16);
+    for (int i = 0; i < 32; ++i) {
+      const uint32_t word = v[i >> 1];
+      const float x = (i & 1) ? __uint_as_float(word & 0xFFFF0000u) : __uint_as_float(word << 16);
       const float r = __fmul_rn(x, inv);
       // |r| <= 8 here: adding 1.5 * 2^23 rounds r to an integer n (nearest, ties to even, as
       // rint) and leaves 2^22 + n in the fraction bits, so u = n + 8 is (bits + 8) mod 2^23
@@ -141,58 +130,64 @@ __device__ __forceinline__ int search_fast_quad(const uint32_t (&v)[4], float a,
       const uint32_t u = __float_as_uint(tr) + 8u - 0x4B400000u;
       dmax = fmaxf(dmax, fabsf(__fsub_rn(r, qf)));
       ubits |= u;                                  // u = 16 (n = +8) is the only way out of range
-      t |= (u & 15u) << nibble_shift(i);
+      t[i >> 3] |= (u & 15u) << nibble_shift(i);
       // least-squares sums of this candidate (exact: see the caller)
-      ps = __fmaf_rn(x, qf, ps);
+      ps[i >> 3] = __fmaf_rn(x, qf, ps[i >> 3]);
       qs = __fmaf_rn(qf, qf, qs);
     }
-    uint32_t fail = (dmax > tol + band) | ((ubits & ~15u) != 0);
-    uint32_t unsure = dmax > tol - band;
-    fail = quad_or(fail, qm);
-    unsure = quad_or(unsure, qm);
+    const bool fail = (dmax > tol + band) || ((ubits & ~15u) != 0);
+    const bool unsure = dmax > tol - band;
     if (!done) {
       if (!fail) {
         done = true;
-        if (!unsure) { result = next; cw = t; psum = ps; qsum = qs; }   // else 0: exact path
+        if (!unsure) {                             // else 0: exact path
+          result = next;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) cw[j] = t[j];
+          // On the grid every nonzero product w q lies within a factor 70 of the others and
+          // carries at most 12 significant bits, so sums of them are exact in any order: eight
+          // in float32 (at most about 21 bits wide), the four partial sums in float64.  This is
+          // the float64 index-order sum of the rule, bit for bit.  sum q^2 <= 2048 is exact too.
+          num = __dadd_rn(__dadd_rn(static_cast<double>(ps[0]), static_cast<double>(ps[1])),
+                          __dadd_rn(static_cast<double>(ps[2]), static_cast<double>(ps[3])));
+          den = static_cast<int>(qs);
+        }
       } else {
         ++next;
         while (next <= 8 && skip(next)) ++next;
-        done = next > 8;                               // off the grid: decided exactly
+        done = next > 8;                           // off the grid: decided exactly
       }
     }
   }
   return result;
 }
 
-// The exact rule (and the off-grid fallback) for a quad's group, run by the quad's first lane on
-// the whole group, with the float64 sum in index order; results broadcast to the quad.  Kept out
-// of line so that the common path's register budget stays small.
-__device__ __noinline__ void exact_quad(const uint32_t (&v)[4], float a, unsigned qm, int qbase,
-                                        int sub, int& m, double& num, int& den, uint32_t& cw) {
+// The exact rule (and the off-grid fallback) for one group, with the float64 sum in index order.
+// Kept out of line so that the common path's register budget stays small.
+__device__ __noinline__ int exact_group(const uint32_t (&v)[16], float a, double& num, int& den,
+                                        uint32_t (&cw)[4]) {
   GroupBits G;
 #pragma unroll
-  for (int k = 0; k < 4; ++k)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) G.v[4 * k + j] = __shfl_sync(qm, v[j], qbase + k);
+  for (int j = 0; j < 16; ++j) G.v[j] = v[j];
   uint32_t cws[4] = {0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u};
-  int mm = 0, dd = 0;
+  const int m = search_exact(G, static_cast<double>(a), cws);
   double nn = 0.0;
-  if (sub == 0) {
-    mm = search_exact(G, static_cast<double>(a), cws);
-    for (int i = 0; i < 32; ++i) {
-      const int qi = code_of(cws, i);
-      nn = __fma_rn(static_cast<double>(elem_f32(G, i)), static_cast<double>(qi), nn);
-      dd += qi * qi;
-    }
+  int dd = 0;
+  for (int i = 0; i < 32; ++i) {
+    const int qi = code_of(cws, i);
+    nn = __fma_rn(static_cast<double>(elem_f32(G, i)), static_cast<double>(qi), nn);
+    dd += qi * qi;
   }
-  m = __shfl_sync(qm, mm, qbase);
-  num = __shfl_sync(qm, nn, qbase);
-  den = __shfl_sync(qm, dd, qbase);
+  num = nn;
+  den = dd;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const uint32_t c = __shfl_sync(qm, cws[k], qbase);
-    if (sub == k) cw = c;
-  }
+  for (int j = 0; j < 4; ++j) cw[j] = cws[j];
+  return m;
+}
+
+__device__ __forceinline__ void load_group(const uint4* __restrict__ w, int64_t gi, uint4 (&u)[4]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) u[j] = __ldg(w + gi * 4 + j);
 }
 
 __global__ void __launch_bounds__(256, 4) repack_kernel(const uint4* __restrict__ w, int64_t groups,
@@ -200,25 +195,27 @@ __global__ void __launch_bounds__(256, 4) repack_kernel(const uint4* __restrict_
                                                      uint16_t* __restrict__ scales,
                                                      uint8_t* __restrict__ group_m,
                                                      unsigned long long* off_grid_count) {
-  const int lane = threadIdx.x & 31, sub = lane & 3, qbase = lane & ~3;
-  const unsigned qm = 0xFu << qbase;
-  const int64_t stride = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 2;
-  for (int64_t gi = ((static_cast<int64_t>(blockIdx.x) * blockDim.x) + threadIdx.x) >> 2; gi < groups;
-       gi += stride) {
-    const uint4 u = ldg_stream128(w + gi * 4 + sub);
-    const uint32_t v[4] = {u.x, u.y, u.z, u.w};
-    uint32_t amax = 0, amin = 0x7FFFu, nonfinite = 0;     // largest and smallest nonzero |w|
+  const int lane = threadIdx.x & 31;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t gi = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  uint4 nx[4];
+  if (gi < groups) load_group(w, gi, nx);
+  for (; gi < groups; gi += stride) {
+    uint32_t v[16];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
+      v[4 * j] = nx[j].x; v[4 * j + 1] = nx[j].y; v[4 * j + 2] = nx[j].z; v[4 * j + 3] = nx[j].w;
+    }
+    if (gi + stride < groups) load_group(w, gi + stride, nx);   // in flight while this one is decided
+    uint32_t amax = 0, amin = 0x7FFFu, nonfinite = 0;          // largest and smallest nonzero |w|
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
       const uint32_t lo = v[j] & 0x7FFFu, hi = (v[j] >> 16) & 0x7FFFu;
       amax = max(amax, max(lo, hi));
       amin = min(amin, min(lo ? lo : 0x7FFFu, hi ? hi : 0x7FFFu));
       nonfinite |= ((lo & 0x7F80u) == 0x7F80u) | ((hi & 0x7F80u) == 0x7F80u);
     }
-    amax = quad_max(amax, qm);
-    amin = quad_min(amin, qm);
-    nonfinite = quad_or(nonfinite, qm);
-    uint32_t cw = 0x88888888u;                            // q = 0
+    uint32_t cw[4] = {0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u};   // q = 0
     int m;
     uint16_t scale_bits;
     bool off = false;
@@ -232,36 +229,22 @@ __global__ void __launch_bounds__(256, 4) repack_kernel(const uint4* __restrict_
     } else {
       const float a = bf16_lo_to_f32(amax);
       m = 0;
-      float ps = 0.f, qs = 0.f;
-      if (a >= 0x1p-100f && a <= 0x1p100f) m = search_fast_quad(v, a, bf16_lo_to_f32(amin), qm, cw, ps, qs);
       double num = 0.0;
       int den = 0;
-      if (m > 0) {
-        // On the grid every nonzero product w q lies within a factor 70 of the others and carries
-        // at most 12 significant bits, so sums of them are exact in any order: a lane's eight in
-        // float32 (at most about 21 bits wide), the quad's four partial sums in float64.  This is
-        // the float64 index-order sum of the rule, bit for bit.  sum q^2 <= 2048 is exact too.
-        num = static_cast<double>(ps);
-        num = __dadd_rn(num, __shfl_xor_sync(qm, num, 1));
-        num = __dadd_rn(num, __shfl_xor_sync(qm, num, 2));
-        den = static_cast<int>(qs);
-        den += __shfl_xor_sync(qm, den, 1);
-        den += __shfl_xor_sync(qm, den, 2);
-      } else {
-        exact_quad(v, a, qm, qbase, sub, m, num, den, cw);
+      if (a >= 0x1p-100f && a <= 0x1p100f) m = search_fast(v, a, bf16_lo_to_f32(amin), cw, num, den);
+      if (m == 0) {
+        m = exact_group(v, a, num, den, cw);
         off = (m == 0);
       }
       const double s = den > 0 ? __ddiv_rn(num, static_cast<double>(den)) : 0.0;
       scale_bits = f64_to_bf16_rne(s);
     }
-    codes[gi * 4 + sub] = cw;
-    if (sub == 0) {
-      scales[gi] = scale_bits;
-      if (group_m) group_m[gi] = static_cast<uint8_t>(m);
-    }
+    reinterpret_cast<uint4*>(codes)[gi] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    scales[gi] = scale_bits;
+    if (group_m) group_m[gi] = static_cast<uint8_t>(m);
     if (off_grid_count) {
       const unsigned active = __activemask();
-      const unsigned ballot = __ballot_sync(active, off && sub == 0);
+      const unsigned ballot = __ballot_sync(active, off);
       if (ballot && lane == __ffs(active) - 1)
         atomicAdd(off_grid_count, static_cast<unsigned long long>(__popc(ballot)));
     }
@@ -279,8 +262,8 @@ w4_status w4_launch_repack(const uint16_t* w, int64_t groups, uint32_t* codes, u
       return W4_ERR_CUDA;
   }
   if (groups == 0) return W4_OK;
-  const int threads = 256;                               // 64 groups per block (four lanes each)
-  int64_t blocks = (groups + 63) / 64;
+  const int threads = 256;                               // 256 groups per block (one lane each)
+  int64_t blocks = (groups + 255) / 256;
   const int64_t cap = static_cast<int64_t>(sm_count) * 16;
   if (blocks > cap) blocks = cap;
   w4::repack_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
