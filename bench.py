@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", choices=list(WORKLOADS), default="moe_decode")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--stack-layers", type=int, default=30,
+                    help="layers of the secondary repack + expert-stack measurement (30: the full stack)")
     ap.add_argument("--seed", type=int, default=0)
     return ap.parse_args()
 
@@ -507,7 +509,7 @@ def run_secondary(args, device, stream):
                                             "frac_bf16_peak": round(flops / ms / 1e9 / tc_peak, 3)}
         del lay
         torch.cuda.empty_cache()
-    out.update(run_stack(device, stream))
+    out.update(run_stack(device, stream, L=args.stack_layers))
     return out
 
 
@@ -534,7 +536,7 @@ def run_stack(device, stream, L=30, reps=3):
     ms = e0.elapsed_time(e1) / reps
     groups = (st.gate_up_rows() * H + st.down_rows() * I) // 32
     moved = groups * (64 + 16 + 2 + 1)          # bf16 in; codes, scale, group_m out
-    res["repack_30x128_experts"] = {"ms": round(ms, 3), "groups": groups, "GB/s": round(moved / ms / 1e6, 1),
+    res[f"repack_{L}x128_experts"] = {"ms": round(ms, 3), "groups": groups, "GB/s": round(moved / ms / 1e6, 1),
                                     "frac_hbm": round(moved / ms / 1e6 / hbm_peak, 3),
                                     "off_grid": rep.off_grid_gate_up + rep.off_grid_down}
     del w_gu, w_dn, rep
@@ -561,7 +563,7 @@ def run_stack(device, stream, L=30, reps=3):
         stream.synchronize()
         ms = e0.elapsed_time(e1) / n
         byts = hit * st.expert_bytes() + L * T * H * 2 * 2
-        res[f"stack_decode_30_layers_T{T}"] = {"ms_per_step": round(ms, 3), "tokens/s": round(T / ms * 1e3, 1),
+        res[f"stack_decode_{L}_layers_T{T}"] = {"ms_per_step": round(ms, 3), "tokens/s": round(T / ms * 1e3, 1),
                                                "experts_hit": hit, "GB/s": round(byts / ms / 1e6, 1),
                                                "frac_hbm": round(byts / ms / 1e6 / hbm_peak, 3)}
         del g

@@ -99,7 +99,7 @@ __device__ __noinline__ int search_exact(const GroupBits& g, double a, uint32_t 
 // skipped without looking at the elements (margins of 2^-16 cover the float32 error of
 // m * wmin / a); on the grid this makes the group's own m the first candidate.  The search runs
 // in rounds over the whole warp: each round every undecided group tries its next candidate.
-__device__ __forceinline__ int search_fast(const uint32_t (&v)[16], float a, float wmin,
+__device__ __forceinline__ int search_fast(const uint32_t (&v)[16], float a, float wmin, float xp,
                                            uint32_t (&cw)[4], double& num, int& den) {
   const float tol = 0.0625f, band = 0x1p-17f, kRound = 12582912.0f;
   const float ra = __frcp_rn(a);
@@ -115,7 +115,7 @@ __device__ __forceinline__ int search_fast(const uint32_t (&v)[16], float a, flo
   const unsigned active = __activemask();
   while (__any_sync(active, !done)) {
     const float inv = __fmul_rn(static_cast<float>(next <= 8 ? next : 8), ra);
-    uint32_t t[4] = {0u, 0u, 0u, 0u}, ubits = 0;
+    uint32_t t[4] = {0u, 0u, 0u, 0u};
     float dmax = 0.f, qs = 0.f;
     float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -129,13 +129,15 @@ __device__ __forceinline__ int search_fast(const uint32_t (&v)[16], float a, flo
       const float qf = __fsub_rn(tr, kRound);
       const uint32_t u = __float_as_uint(tr) + 8u - 0x4B400000u;
       dmax = fmaxf(dmax, fabsf(__fsub_rn(r, qf)));
-      ubits |= u;                                  // u = 16 (n = +8) is the only way out of range
-      t[i >> 3] |= (u & 15u) << nibble_shift(i);
+      t[i >> 3] += u << nibble_shift(i);           // disjoint fields while every u <= 15
       // least-squares sums of this candidate (exact: see the caller)
       ps[i >> 3] = __fmaf_rn(x, qf, ps[i >> 3]);
       qs = __fmaf_rn(qf, qf, qs);
     }
-    const bool fail = (dmax > tol + band) || ((ubits & ~15u) != 0);
+    // u = 16 (n = +8) is the only way out of range.  x -> rint(x * inv) is monotonic, so it
+    // happens exactly when it happens for the largest element xp (the same float32 operations)
+    const uint32_t up = __float_as_uint(__fadd_rn(__fmul_rn(xp, inv), kRound)) + 8u - 0x4B400000u;
+    const bool fail = (dmax > tol + band) || up > 15u;
     const bool unsure = dmax > tol - band;
     if (!done) {
       if (!fail) {
@@ -207,14 +209,25 @@ __global__ void __launch_bounds__(256, 4) repack_kernel(const uint4* __restrict_
       v[4 * j] = nx[j].x; v[4 * j + 1] = nx[j].y; v[4 * j + 2] = nx[j].z; v[4 * j + 3] = nx[j].w;
     }
     if (gi + stride < groups) load_group(w, gi + stride, nx);   // in flight while this one is decided
-    uint32_t amax = 0, amin = 0x7FFFu, nonfinite = 0;          // largest and smallest nonzero |w|
+    // Largest and smallest nonzero |w| (bf16 magnitude bits), and the largest element, two
+    // elements per instruction: |w| - 1 per half-word (zero -> 0xFFFF) is (y + 0x7FFF) ^ 0x8000
+    // for y <= 0x7FFF, with no carry between the halves; bf16 bit patterns compared as signed
+    // 16-bit integers order the non-negative values (and any non-negative one beats every
+    // negative one).
+    uint32_t amax2 = 0u, zmin2 = 0xFFFFFFFFu, pmax2 = 0x80008000u;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      const uint32_t lo = v[j] & 0x7FFFu, hi = (v[j] >> 16) & 0x7FFFu;
-      amax = max(amax, max(lo, hi));
-      amin = min(amin, min(lo ? lo : 0x7FFFu, hi ? hi : 0x7FFFu));
-      nonfinite |= ((lo & 0x7F80u) == 0x7F80u) | ((hi & 0x7F80u) == 0x7F80u);
+      const uint32_t y = v[j] & 0x7FFF7FFFu;
+      amax2 = __vmaxu2(amax2, y);
+      zmin2 = __vminu2(zmin2, (y + 0x7FFF7FFFu) ^ 0x80008000u);
+      pmax2 = __vmaxs2(pmax2, v[j]);
     }
+    const uint32_t amax = max(amax2 & 0xFFFFu, amax2 >> 16);
+    const uint32_t zmin = min(zmin2 & 0xFFFFu, zmin2 >> 16);
+    const uint32_t amin = zmin == 0xFFFFu ? 0x7FFFu : zmin + 1u;
+    const bool nonfinite = amax >= 0x7F80u;                    // exponent all ones: inf or NaN
+    const int16_t p_lo = static_cast<int16_t>(pmax2 & 0xFFFFu), p_hi = static_cast<int16_t>(pmax2 >> 16);
+    const uint32_t pbits = static_cast<uint16_t>(p_lo > p_hi ? p_lo : p_hi);
     uint32_t cw[4] = {0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u};   // q = 0
     int m;
     uint16_t scale_bits;
@@ -231,7 +244,8 @@ __global__ void __launch_bounds__(256, 4) repack_kernel(const uint4* __restrict_
       m = 0;
       double num = 0.0;
       int den = 0;
-      if (a >= 0x1p-100f && a <= 0x1p100f) m = search_fast(v, a, bf16_lo_to_f32(amin), cw, num, den);
+      if (a >= 0x1p-100f && a <= 0x1p100f)
+        m = search_fast(v, a, bf16_lo_to_f32(amin), bf16_lo_to_f32(pbits), cw, num, den);
       if (m == 0) {
         m = exact_group(v, a, num, den, cw);
         off = (m == 0);
