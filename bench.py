@@ -7,10 +7,10 @@ bf16 scales).  A step is one pass of the hot path: route + permute, gate/up grou
 GELU gate, down grouped GEMM, weighted combine.  Metric: tokens per second (higher is better).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
-                  [--workload moe_decode|moe_prefill] [--no-secondary]
+                  [--workload moe_decode|moe_prefill] [--no-secondary] [--stack-layers L]
 
-Multi-GPU: the layer does not shard in this build; N ranks run N independent replicas (weak
-scaling), timed on the device with the max over ranks.  `--impl reference` times the CPU oracle
+Multi-GPU: the layer does not shard; N ranks run N independent replicas (weak scaling, no
+data-path collective), timed on the device with the max over ranks.  `--impl reference` times the CPU oracle
 (the correctness reference) on the same workload, one token per step.
 """
 from __future__ import annotations
@@ -60,6 +60,48 @@ def dist_setup(n_gpus):
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def ranks_init(world, backend="nccl", device=None, timeout_s=120):
+    """Join the job's process group (one process per GPU, env:// rendezvous as torchrun sets it
+    up), with a short timeout so that ranks waiting on a lost peer end with an error."""
+    if world <= 1:
+        return
+    import torch.distributed as dist
+    from datetime import timedelta
+    kw = {"timeout": timedelta(seconds=timeout_s)}
+    if device is not None:
+        kw["device_id"] = device
+    dist.init_process_group(backend, **kw)
+
+
+def ranks_barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def ranks_max(x, world, device=None):
+    """The maximum of x over all ranks: a job's device time is its slowest rank's."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, ms):
+    """Whole-job units per second: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / (ms / 1e3)
+
+
+def ranks_finish(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 def peaks():
@@ -200,10 +242,7 @@ def native(args, world, rank, local):
 
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    if world > 1:
-        import torch.distributed as dist
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    ranks_init(world, "nccl", device)
     wl = WORKLOADS[args.workload]
     T, E, k, H, I = wl["T"], 128, 8, 2816, 704
     case = synth.moe_case(T, E, k, H, I, seed=args.seed + rank, zipf_s=wl["zipf"])
@@ -238,9 +277,7 @@ def native(args, world, rank, local):
     gpu_index = _physical_gpu_index(local)
     clocks = ClockSampler(gpu_index)
     clocks.start()
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    ranks_barrier(world)
     torch.cuda.synchronize()
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
@@ -253,16 +290,11 @@ def native(args, world, rank, local):
     stream.synchronize()
     clocks.mark("end")
     torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-        dist.barrier()
+    ms = ranks_max(ev0.elapsed_time(ev1), world, device)
+    ranks_barrier(world)
     clocks.stop()
     ms_per_step = ms / args.steps
-    value = T * world * args.steps / (ms / 1e3)
+    value = job_throughput(T * args.steps, world, ms)
 
     # ---------------- per-kernel durations of the grouped GEMM (same launches) ----------------
     # Each GEMM call (its preparation pass included) replayed from a CUDA graph, alternating the
@@ -348,9 +380,7 @@ def native(args, world, rank, local):
             y = lay(x_d, lg_d)
             y_h.copy_(y, non_blocking=True)
     stream.synchronize()
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    ranks_barrier(world)
     f0 = torch.cuda.Event(enable_timing=True)
     f1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
@@ -362,13 +392,8 @@ def native(args, world, rank, local):
             y_h.copy_(y, non_blocking=True)
         f1.record(stream)
     stream.synchronize()
-    ms_e2e = f0.elapsed_time(f1)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms_e2e], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
-    e2e_value = T * world * n_e2e / (ms_e2e / 1e3)
+    ms_e2e = ranks_max(f0.elapsed_time(f1), world, device)
+    e2e_value = job_throughput(T * n_e2e, world, ms_e2e)
 
     secondary = {}
     if not args.no_secondary and rank == 0:
@@ -378,11 +403,8 @@ def native(args, world, rank, local):
     if rank == 0 and world == 1:
         cpu_base = cpu_baseline(case)
 
-    if world > 1:
-        import torch.distributed as dist
-        del graph
-        dist.barrier()
-        dist.destroy_process_group()
+    del graph                    # (holds no collective) released before the group goes
+    ranks_finish(world)
     if rank != 0:
         return
     line = {
