@@ -24,6 +24,7 @@ Modules:
 
 Where the pages leave a step open, the reading taken is stated in the function's docstring.
 Pins that tie each function to something other than itself live in ``tests/test_oracle_*.py``.
-Parity unpinned: the tanh-GELU gate is not on the pages; it is tied only to mathematical
-identities and to the erf form (see ``moe.gelu_tanh``).
+The tanh-GELU gate is not on the pages (a reading: the tanh form of GELU); ``moe.gelu_tanh`` is
+pinned to mathematical identities, to the erf form, and to PyTorch's tanh-approximate GELU, an
+independent implementation of the same published approximation.
 """

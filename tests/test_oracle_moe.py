@@ -4,9 +4,9 @@ The pages give "128 experts per layer and 8 active per token" ("Repacked QAT Gem
 serves on one TPU v6e at 1.9x FP8 throughput", section "The gap at 26B") and a grouped matmul
 over the experts' packed int4 weights with per-32 scales (section "What changed in vLLM's TPU
 backend").  The router math, the gate/up split and the activation are not on the pages; they
-are pinned here to library routines (softmax, sorting, erf) and to mathematical identities.
-
-Parity unpinned beyond formula agreement: the tanh-GELU gate (no page value exists for it).
+are pinned here to library routines (softmax, sorting, erf, PyTorch's tanh-approximate GELU)
+and to mathematical identities.  No page value exists for the tanh-GELU gate; it is pinned to
+an independent implementation of the same published approximation.
 """
 import math
 
@@ -77,6 +77,16 @@ def test_gelu_identities_and_erf_form():
     erf_form = np.array([0.5 * v * (1 + math.erf(v / math.sqrt(2))) for v in z])
     assert np.max(np.abs(g - erf_form)) < 1e-3
     assert abs(g[-1] - 12) < 1e-9 and abs(g[0]) < 1e-9
+
+
+def test_gelu_matches_an_independent_tanh_gelu():
+    """PyTorch's tanh-approximate GELU, a separate implementation of the same published
+    approximation (Hendrycks and Gimpel's tanh form), agrees in float64; a wrong cubic
+    coefficient or scale would differ by far more than rounding."""
+    import torch
+    z = np.linspace(-12, 12, 20001)
+    ref = torch.nn.functional.gelu(torch.tensor(z, dtype=torch.float64), approximate="tanh").numpy()
+    assert np.max(np.abs(moe.gelu_tanh(z) - ref)) < 1e-13
 
 
 def test_gmm_rows_equal_dense_linear_per_expert():
