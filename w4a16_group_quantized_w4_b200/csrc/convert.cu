@@ -105,6 +105,78 @@ row_exp_kernel(const uint16_t* __restrict__ scales, int64_t wrows, int kg, int8_
   }
 }
 
+// Short rows (at most 128 16-byte chunks, K <= 1024): a warp converts 12 / CPL rows at a time,
+// lane l holding chunks l + 32 t (t < CPL) of each, so that twelve loads per lane are in flight
+// as for long rows (one row per warp would leave a K = 704 row at three).  Same arithmetic as
+// a_to_f16_kernel.
+template <int CPL>
+__global__ void __launch_bounds__(256)
+a_to_f16_short_kernel(const uint16_t* __restrict__ a, const int32_t* __restrict__ a_row_of_pair,
+                      int k_div, int64_t a_rows, int64_t rows, int K, uint16_t* __restrict__ a16,
+                      float* __restrict__ rowmul, int32_t* dev_status) {
+  constexpr int kRW = 12 / CPL;
+  const int lane = threadIdx.x & 31;
+  const int64_t wpb = blockDim.x >> 5;
+  const int nv = K >> 3;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * wpb;
+  for (int64_t r0 = (blockIdx.x * wpb + (threadIdx.x >> 5)) * kRW; r0 < rows; r0 += nw * kRW) {
+    uint4 v[kRW][CPL];
+#pragma unroll
+    for (int j = 0; j < kRW; ++j) {
+      const int64_t row = r0 + j;
+      int64_t srow = row;
+      if (row < rows && a_row_of_pair) {
+        srow = __ldg(a_row_of_pair + row) / k_div;
+        if (srow < 0 || srow >= a_rows) {
+          if (lane == 0) set_status(dev_status, W4_ERR_INVALID_ARG);
+          srow = 0;
+        }
+      }
+      const uint4* src = reinterpret_cast<const uint4*>(a + srow * K);
+#pragma unroll
+      for (int t = 0; t < CPL; ++t) {
+        const int i = 32 * t + lane;
+        v[j][t] = (row < rows && i < nv) ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kRW; ++j) {
+      const int64_t row = r0 + j;
+      uint32_t m = 0;
+#pragma unroll
+      for (int t = 0; t < CPL; ++t) {
+        const uint32_t w[4] = {v[j][t].x, v[j][t].y, v[j][t].z, v[j][t].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t lo = w[q] & 0x7FFFu, hi = (w[q] >> 16) & 0x7FFFu;
+          if (lo < 0x7F80u) m = max(m, lo);
+          if (hi < 0x7F80u) m = max(m, hi);
+        }
+      }
+      m = __reduce_max_sync(0xffffffffu, m);
+      if (row >= rows) continue;                 // the same for every lane of the warp
+      const int f = shift_for(m, 14);
+      const float mul = pow2f(f);
+      uint4* dst = reinterpret_cast<uint4*>(a16 + row * K);
+#pragma unroll
+      for (int t = 0; t < CPL; ++t) {
+        const int i = 32 * t + lane;
+        if (i < nv) {
+          const uint32_t w[4] = {v[j][t].x, v[j][t].y, v[j][t].z, v[j][t].w};
+          uint32_t o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const __half2 h = __floats2half2_rn(bf16_lo_to_f32(w[q]) * mul, bf16_hi_to_f32(w[q]) * mul);
+            o[q] = *reinterpret_cast<const uint32_t*>(&h);
+          }
+          dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+      if (lane == 0) rowmul[row] = pow2f(-f);
+    }
+  }
+}
+
 }  // namespace cv
 }  // namespace w4
 
@@ -132,11 +204,28 @@ void w4_launch_a_to_f16(const uint16_t* a, const int32_t* a_row_of_pair, int k_d
                         int64_t rows, int K, const uint16_t* scales, int64_t wrows, void* ws,
                         int32_t* dev_status, cudaStream_t stream, int sm_count) {
   if (rows <= 0) return;
-  const int64_t blocks = (rows + 7) / 8;
-  const int grid = static_cast<int>(blocks < 16LL * sm_count ? blocks : 16LL * sm_count);
-  w4::cv::a_to_f16_kernel<<<grid, 256, 0, stream>>>(a, a_row_of_pair, k_div, a_rows, rows, K,
-                                                    w4_ws_a16(ws), w4_ws_rowmul(ws, rows, K),
-                                                    dev_status);
+  const int nv = K >> 3;
+  if (nv <= 128) {
+    // short rows: 12 / cpl rows per warp at a time
+    const int cpl = (nv + 31) / 32;
+    const int64_t warps = (rows + 12 / cpl - 1) / (12 / cpl);
+    const int64_t blocks = (warps + 7) / 8;
+    const int grid = static_cast<int>(blocks < 16LL * sm_count ? blocks : 16LL * sm_count);
+    uint16_t* a16 = w4_ws_a16(ws);
+    float* rm = w4_ws_rowmul(ws, rows, K);
+    switch (cpl) {
+      case 1: w4::cv::a_to_f16_short_kernel<1><<<grid, 256, 0, stream>>>(a, a_row_of_pair, k_div, a_rows, rows, K, a16, rm, dev_status); break;
+      case 2: w4::cv::a_to_f16_short_kernel<2><<<grid, 256, 0, stream>>>(a, a_row_of_pair, k_div, a_rows, rows, K, a16, rm, dev_status); break;
+      case 3: w4::cv::a_to_f16_short_kernel<3><<<grid, 256, 0, stream>>>(a, a_row_of_pair, k_div, a_rows, rows, K, a16, rm, dev_status); break;
+      default: w4::cv::a_to_f16_short_kernel<4><<<grid, 256, 0, stream>>>(a, a_row_of_pair, k_div, a_rows, rows, K, a16, rm, dev_status); break;
+    }
+  } else {
+    const int64_t blocks = (rows + 7) / 8;
+    const int grid = static_cast<int>(blocks < 16LL * sm_count ? blocks : 16LL * sm_count);
+    w4::cv::a_to_f16_kernel<<<grid, 256, 0, stream>>>(a, a_row_of_pair, k_div, a_rows, rows, K,
+                                                      w4_ws_a16(ws), w4_ws_rowmul(ws, rows, K),
+                                                      dev_status);
+  }
   if (wrows > 0) {
     const int64_t eb = (wrows + 255) / 256;
     const int egrid = static_cast<int>(eb < 8LL * sm_count ? eb : 8LL * sm_count);
