@@ -19,11 +19,12 @@
  *     default stream).  Nothing synchronises the host and nothing is copied to the host.
  *   - bf16 values are passed as their uint16 bit patterns.  Arrays are dense and row-major.
  *   - Packed codes ("layout L1"): a row of K weights is K/8 uint32 words holding u = q + 8 (q is
- *     the int4 code in -8..7) of elements 8w..8w+7: bits 4i..4i+3 of word w hold element 8w + 2i
- *     and bits 16+4i..16+4i+3 hold element 8w + 2i + 1, i = 0..3 (even elements in the low
- *     half-word, odd in the high).  Four consecutive words (16 bytes) hold exactly one group of
- *     32, so one 16-byte load is one group.  Scales are one bf16 per
- *     group: scales[r][g] scales elements 32g..32g+31 of row r.  Dequantised weight = s * q.
+ *     the int4 code in -8..7) of elements 8w..8w+7 in k order: bits 4j..4j+3 of word w hold
+ *     element 8w + j, j = 0..7 (the lowest nibble is the lowest k).  Four consecutive words
+ *     (16 bytes) hold exactly one group of 32, so one 16-byte load is one group.  The kernels
+ *     read this layout as it is; any reordering they need happens on the activation side.
+ *     Scales are one bf16 per group: scales[r][g] scales elements 32g..32g+31 of row r.
+ *     Dequantised weight = s * q.
  *   - The returned status reports host-side checks (null pointers, sizes, alignment) and launch
  *     failures (W4_ERR_CUDA; the CUDA error is available from w4_last_cuda_error()).  Conditions
  *     found on the device are written to the optional `dev_status` word, which the caller reads

@@ -22,11 +22,10 @@ Readings taken where the pages are open (each is also listed in the design notes
   * an all-zero group has scale 0, codes 0 and m = 1; a group holding NaN or infinity is
     off the grid with codes 0 and a NaN scale.
 
-Packed layout (ours; the container's bit layout is not on the pages): codes[r, w] is a uint32
-holding u = q + 8 of elements k = 8w .. 8w+7: bits 4i..4i+3 hold element 8w + 2i and bits
-16+4i..16+4i+3 hold element 8w + 2i + 1, for i = 0..3 (even elements in the low half-word, odd
-elements in the high half-word, each in k order).  One 16-byte run of four words is exactly one
-group of 32.  Scales[r, g] is the bf16 scale of elements 32g..32g+31 of row r.
+Packed layout L1 (ours; the container's bit layout is not on the pages): codes[r, w] is a
+uint32 holding u = q + 8 of elements k = 8w .. 8w+7 in k order: bits 4j..4j+3 hold element
+8w + j, j = 0..7 (the lowest nibble is the lowest k).  One 16-byte run of four words is exactly
+one group of 32.  Scales[r, g] is the bf16 scale of elements 32g..32g+31 of row r.
 """
 from __future__ import annotations
 
@@ -47,8 +46,8 @@ REPRODUCE_TOL = 1.0 / 16.0
 # ------------------------------------------------------------------------------------------
 
 def nibble_shift(j: int) -> int:
-    """Bit offset of element 8w + j inside word w: even j in the low half-word, odd j in the high."""
-    return 4 * (j // 2) + (16 if j % 2 else 0)
+    """Bit offset of element 8w + j inside word w (layout L1: nibble j holds element j)."""
+    return 4 * j
 
 
 def pack(q) -> np.ndarray:

@@ -93,3 +93,38 @@ def test_workspace_reused_across_shapes_with_stale_contents():
         cols = np.arange(0, N, 97)
         ref = linear.w4a16_linear_rows(case.x, case.codes, case.scales, cols)
         assert_rows_close(host_f64(y)[:, cols], ref)
+
+
+def _golden_words():
+    """(codes q_0..q_7, word) pairs worked by hand in tests/golden/nibble_layout.txt (layout L1)."""
+    import os
+    out = []
+    for line in open(os.path.join(os.path.dirname(__file__), "golden", "nibble_layout.txt")):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        lhs, rhs = line.split("->")
+        out.append(([int(v) for v in lhs.split()], int(rhs, 16)))
+    return out
+
+
+@pytest.mark.parametrize("M", [16, 64])          # weight-streaming kernel, tensor-core kernel
+def test_golden_l1_words_through_linear(M):
+    """Hand-packed layout-L1 words (not produced by the oracle) as the weights of a linear with
+    scale 1 and one-hot activation rows: y[m, n] must be exactly code m of row n, as the golden
+    file lists it.  A kernel that read the nibbles in any other order fails this bit for bit."""
+    gold = _golden_words()
+    N, K = 128, 64
+    words = np.empty((N, K // 8), np.uint32)
+    q = np.empty((N, K), np.int64)
+    for n in range(N):
+        for w in range(K // 8):
+            codes, word = gold[(n * 3 + w) % len(gold)]
+            words[n, w] = word
+            q[n, 8 * w:8 * w + 8] = codes
+    x = np.eye(K, dtype=np.float32)[np.arange(M) % K]
+    s_bits = synth.f32_to_bf16_bits(np.ones((N, K // 32), np.float32))
+    y = api.w4a16_linear(dev_bf16(synth.f32_to_bf16_bits(x)), dev_u32(words), dev_bf16(s_bits))
+    torch.cuda.synchronize()
+    expect = q[:, np.arange(M) % K].T.astype(np.float64)
+    assert np.array_equal(host_f64(y), expect)

@@ -75,7 +75,7 @@ def test_brute_force_loops_with_hand_decoded_nibbles():
             for k in range(K):
                 word = int(words[n, k // 8])
                 j = k % 8
-                u = (word >> (4 * (j // 2) + 16 * (j % 2))) & 0xF   # even j low half, odd j high
+                u = (word >> (4 * j)) & 0xF                        # layout L1: nibble j = element j
                 acc += xf[m][k] * float(sf[n, k // 32]) * (u - 8)
             assert abs(acc - y[m, n]) <= 1e-12 * (1 + abs(acc))
 

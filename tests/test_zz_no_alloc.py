@@ -70,3 +70,24 @@ def test_noalloc_rejects_a_row_beyond_its_scratch():
     p = C.c_void_p(dummy.data_ptr())
     status = lib.w4a16_linear_noalloc(p, p, p, p, M, N, K, C.c_void_p(None))
     assert status == _lib.W4_ERR_WORKSPACE
+
+
+def test_noalloc_last_chunk_that_needs_more_scratch_than_the_others():
+    """289 rows against N = 2048, K = 16384: the rows run in chunks, and the shorter last chunk
+    makes fewer work units, so it can split K and need float32 partials that the longer chunks
+    do not.  The call must size its chunks so that every launch fits the 8 MiB array and match
+    the regular entry point on every row."""
+    lib = _lib.load()
+    M, N, K = 289, 2048, 16384
+    case = synth.dense_case(M, N, K, 0.01, 1e-4, seed=13)
+    x, codes, scales = dev_bf16(case.x), dev_u32(case.codes), dev_bf16(case.scales)
+    ref = host_f64(api.w4a16_linear(x, codes, scales))
+    for _ in range(2):
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        st = C.c_void_p(torch.cuda.current_stream().cuda_stream)
+        status = lib.w4a16_linear_noalloc(C.c_void_p(x.data_ptr()), C.c_void_p(codes.data_ptr()),
+                                          C.c_void_p(scales.data_ptr()), C.c_void_p(y.data_ptr()),
+                                          M, N, K, st)
+        assert status == _lib.W4_OK, lib.w4_status_str(status)
+        torch.cuda.synchronize()
+        assert_rows_close(host_f64(y), ref)

@@ -67,6 +67,9 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 }  // namespace
 
+// Status recording for entry points defined in other files of the library.
+w4_status w4_record_status(w4_status s) { return finish(s); }
+
 extern "C" {
 
 const char* w4_status_str(int32_t s) {

@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "../../include/w4a16.h"
@@ -201,6 +202,24 @@ __device__ __forceinline__ uint32_t nib_f16x2_hi(uint32_t v) {   // bits 4..7 | 
   uint32_t r;
   asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(v), "r"(0x00F000F0u), "r"(0x64006400u));
   return r;
+}
+
+// k order of the kernels' extracted fp16 pairs.  Both GEMMs split a layout-L1 code word (nibble j =
+// element j of eight) into the pairs (0, 4), (1, 5), (2, 6), (3, 7): one mask takes the nibbles at
+// bits 4j and 16 + 4j together.  The activation side is written in the same order, so a pair of
+// weights always meets its own pair of activations: eight bf16 values (x0..x7, two per word of w)
+// become four fp16 pairs (x0, x4), (x1, x5), (x2, x6), (x3, x7); the first and third pair are
+// multiplied by m_even, the second and fourth by m_odd.
+__device__ __forceinline__ void f16_pairs_l1(const uint32_t (&w)[4], float m_even, float m_odd,
+                                             uint32_t (&o)[4]) {
+  const __half2 h0 = __floats2half2_rn(bf16_lo_to_f32(w[0]) * m_even, bf16_lo_to_f32(w[2]) * m_even);
+  const __half2 h1 = __floats2half2_rn(bf16_hi_to_f32(w[0]) * m_odd, bf16_hi_to_f32(w[2]) * m_odd);
+  const __half2 h2 = __floats2half2_rn(bf16_lo_to_f32(w[1]) * m_even, bf16_lo_to_f32(w[3]) * m_even);
+  const __half2 h3 = __floats2half2_rn(bf16_hi_to_f32(w[1]) * m_odd, bf16_hi_to_f32(w[3]) * m_odd);
+  o[0] = *reinterpret_cast<const uint32_t*>(&h0);
+  o[1] = *reinterpret_cast<const uint32_t*>(&h1);
+  o[2] = *reinterpret_cast<const uint32_t*>(&h2);
+  o[3] = *reinterpret_cast<const uint32_t*>(&h3);
 }
 
 // D = A(16x16 fp16, row) * B(16x8 fp16, col) + C, float32 accumulators.

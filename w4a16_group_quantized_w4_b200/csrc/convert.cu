@@ -13,6 +13,8 @@ namespace cv {
 // One warp per output row p: the activation row it reads (row p of `a`, or row
 // a_row_of_pair[p] / k_div when rows are gathered) is scanned for its largest finite |a|, which
 // picks f so that it lands in [2^14, 2^15); row p of a16 becomes fp16(a * 2^f) and rowmul[p] = 2^-f.
+// Within every 8 consecutive k the values are stored in the order 0, 4, 1, 5, 2, 6, 3, 7: the
+// order in which the GEMM extracts the nibbles of a layout-L1 code word.
 // A bf16 value of magnitude at least 2^-17 is a multiple of 2^-24 with 8 significant bits, so fp16
 // holds it exactly: every element within a factor 2^31 of the row's largest converts exactly,
 // smaller ones round to the fp16 subnormal grid.  Infinities and NaNs pass through as fp16 inf /
@@ -74,11 +76,7 @@ a_to_f16_kernel(const uint16_t* __restrict__ a, const int32_t* __restrict__ a_ro
         if (i >= nv) break;
         const uint32_t w[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
         uint32_t o[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const __half2 h = __floats2half2_rn(bf16_lo_to_f32(w[j]) * mul, bf16_hi_to_f32(w[j]) * mul);
-          o[j] = *reinterpret_cast<const uint32_t*>(&h);
-        }
+        f16_pairs_l1(w, mul, mul, o);            // k order of the dequantised weight pairs
         dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
@@ -164,11 +162,7 @@ a_to_f16_short_kernel(const uint16_t* __restrict__ a, const int32_t* __restrict_
         if (i < nv) {
           const uint32_t w[4] = {v[j][t].x, v[j][t].y, v[j][t].z, v[j][t].w};
           uint32_t o[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const __half2 h = __floats2half2_rn(bf16_lo_to_f32(w[q]) * mul, bf16_hi_to_f32(w[q]) * mul);
-            o[q] = *reinterpret_cast<const uint32_t*>(&h);
-          }
+          f16_pairs_l1(w, mul, mul, o);
           dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
         }
       }

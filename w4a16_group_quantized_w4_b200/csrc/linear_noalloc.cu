@@ -52,7 +52,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 
 }  // namespace
 
-// from stream_gemm.cu / api.cu
+// from stream_gemm.cu / api.cu (w4_record_status: records the CUDA error behind a W4_ERR_CUDA
+// for w4_last_cuda_error, as every other entry point does)
+w4_status w4_record_status(w4_status s);
 size_t w4_stream_workspace_bytes(int64_t rows, int N, int K, int E, int epi, bool dense, int sm_count);
 w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int k_div,
                                 const uint32_t* codes, const uint16_t* scales,
@@ -74,19 +76,27 @@ w4_status w4a16_linear_noalloc(const uint16_t* x, const uint32_t* codes, const u
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return W4_ERR_CUDA;
+    return w4_record_status(W4_ERR_CUDA);
   // rows in chunks whose workspace (prepared activation rows, split-K partials) fits the scratch
   auto need_for = [&](int64_t rows) {
     return w4_stream_workspace_bytes(rows, static_cast<int>(N), static_cast<int>(K), 1, W4_EPI_NONE,
                                      true, sms);
   };
   if (M == 0) return W4_OK;
+  // The scratch a launch needs is not monotonic in its row count: fewer rows make fewer work
+  // units, which can split K and add float32 partials.  So every row count that will actually
+  // be launched -- the chunk and the shorter last chunk -- must fit before anything runs.
+  if (need_for(1) > kNoallocScratchBytes) return W4_ERR_WORKSPACE;   // one row is too large
+  auto fits = [&](int64_t c) {
+    const int64_t tail = M % c;
+    return need_for(c) <= kNoallocScratchBytes && (tail == 0 || need_for(tail) <= kNoallocScratchBytes);
+  };
   int64_t chunk = M;
   while (chunk > 1 && need_for(chunk) > kNoallocScratchBytes) chunk = (chunk + 1) / 2;
-  if (need_for(chunk) > kNoallocScratchBytes) return W4_ERR_WORKSPACE;   // one row is too large
+  while (chunk > 1 && !fits(chunk)) --chunk;                         // chunk 1 always fits
   cudaError_t err;
   void* ws = scratch_for_current_device(&err);
-  if (!ws) return W4_ERR_CUDA;
+  if (!ws) return w4_record_status(W4_ERR_CUDA);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   for (int64_t r0 = 0; r0 < M; r0 += chunk) {
     const int64_t rows = M - r0 < chunk ? M - r0 : chunk;
@@ -94,7 +104,7 @@ w4_status w4a16_linear_noalloc(const uint16_t* x, const uint32_t* codes, const u
     const w4_status st = w4_launch_stream_gemm(x + r0 * K, nullptr, 1, codes, scales, nullptr, 1, rows,
                                                static_cast<int>(N), static_cast<int>(K), W4_EPI_NONE,
                                                y + r0 * N, ws, kNoallocScratchBytes, nullptr, s, sms);
-    if (st != W4_OK) return st;
+    if (st != W4_OK) return w4_record_status(st);
   }
   return W4_OK;
 }

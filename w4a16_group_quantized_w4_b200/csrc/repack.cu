@@ -51,9 +51,9 @@ __device__ __forceinline__ float elem_f32(const GroupBits& g, int i) {
   return (i & 1) ? bf16_lo_to_f32(g.v[i >> 1] >> 16) : bf16_lo_to_f32(g.v[i >> 1]);
 }
 
-// Bit position of element i's nibble inside code word i / 8 (layout L1: even elements in the low
-// half-word, odd ones in the high half-word, two consecutive k per extracted pair).
-__host__ __device__ constexpr int nibble_shift(int i) { return 4 * ((i & 7) >> 1) + 16 * (i & 1); }
+// Bit position of element i's nibble inside code word i / 8 (layout L1: nibble j of a word holds
+// element j of its eight, in k order).
+__host__ __device__ constexpr int nibble_shift(int i) { return 4 * (i & 7); }
 
 __device__ __forceinline__ int code_of(const uint32_t (&cw)[4], int i) {
   return static_cast<int>((cw[i >> 3] >> nibble_shift(i)) & 15u) - 8;

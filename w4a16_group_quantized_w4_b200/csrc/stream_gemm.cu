@@ -759,15 +759,15 @@ stream_prep_kernel(const uint16_t* __restrict__ a, const int32_t* __restrict__ a
       for (int t = 0; t < kPB; ++t) {
         const int j = j0 + t;
         if (j >= nblk) break;
-        const __half2 h0 = __floats2half2_rn(bf16_lo_to_f32(v[t].x) * m1, bf16_hi_to_f32(v[t].x) * m1);
-        const __half2 h1 = __floats2half2_rn(bf16_lo_to_f32(v[t].y) * m16, bf16_hi_to_f32(v[t].y) * m16);
-        const __half2 h2 = __floats2half2_rn(bf16_lo_to_f32(v[t].z) * m1, bf16_hi_to_f32(v[t].z) * m1);
-        const __half2 h3 = __floats2half2_rn(bf16_lo_to_f32(v[t].w) * m16, bf16_hi_to_f32(v[t].w) * m16);
-        const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
-        const float2 f2 = __half22float2(h2), f3 = __half22float2(h3);
+        const uint32_t w[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
+        uint32_t h[4];
+        f16_pairs_l1(w, m1, m16, h);             // (x0, x4), (x1, x5)/16, (x2, x6), (x3, x7)/16
+        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h[0]));
+        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h[1]));
+        const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&h[2]));
+        const float2 f3 = __half22float2(*reinterpret_cast<const __half2*>(&h[3]));
         float part = 1032.f * ((f0.x + f0.y) + (f2.x + f2.y)) + 1152.f * ((f1.x + f1.y) + (f3.x + f3.y));
-        const uint4 o = make_uint4(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1),
-                                   *reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&h3));
+        const uint4 o = make_uint4(h[0], h[1], h[2], h[3]);
         uint8_t* blk = dst + static_cast<int64_t>(j) * kPrepStage;
         *reinterpret_cast<uint4*>(blk + lane * 16) = o;
         part += __shfl_xor_sync(0xffffffffu, part, 1);

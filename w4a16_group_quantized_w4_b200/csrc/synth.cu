@@ -114,8 +114,8 @@ __global__ void planted_kernel(uint64_t key, int64_t group0, int64_t ngroups, ui
   }
 }
 
-// Groups whose packed codes (4 words per group; in word t, bits 4i..4i+3 hold u = q + 8 of element
-// 8t + 2i and bits 16 + 4i.. those of element 8t + 2i + 1) differ from the planted codes.
+// Groups whose packed codes (4 words per group, layout L1: in word t, bits 4j..4j+3 hold u = q + 8
+// of element 8t + j) differ from the planted codes.
 __global__ void mismatch_kernel(uint64_t key, int64_t group0, int64_t ngroups, const uint32_t* codes,
                                 unsigned long long* count) {
   unsigned long long bad = 0;
@@ -129,10 +129,7 @@ __global__ void mismatch_kernel(uint64_t key, int64_t group0, int64_t ngroups, c
 #pragma unroll
     for (int t = 0; t < 4; ++t)
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        same &= static_cast<int>((cw[t] >> (4 * k)) & 15u) - 8 == G.q[8 * t + 2 * k];
-        same &= static_cast<int>((cw[t] >> (16 + 4 * k)) & 15u) - 8 == G.q[8 * t + 2 * k + 1];
-      }
+      for (int j = 0; j < 8; ++j) same &= static_cast<int>((cw[t] >> (4 * j)) & 15u) - 8 == G.q[8 * t + j];
     bad += same ? 0 : 1;
   }
   for (int o = 16; o; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);

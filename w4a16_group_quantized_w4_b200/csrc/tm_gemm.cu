@@ -190,12 +190,13 @@ __device__ __forceinline__ uint32_t deq_pair(uint32_t v, uint32_t s2, uint32_t c
   return y;
 }
 
-// one code word (eight consecutive k, layout L1) -> four fp16 pairs = four TMEM columns
+// one code word (eight consecutive k, layout L1: nibble j = element j) -> four fp16 pairs = four
+// TMEM columns, in the k order 0, 4, 1, 5, 2, 6, 3, 7 that the conversion pass gives the tokens
 __device__ __forceinline__ void deq_word(uint32_t w, uint32_t s2, uint32_t c2, uint32_t* o) {
-  o[0] = deq_pair(w << 6, s2, c2);   // elements 0, 1 (bits 0-3, 16-19)
-  o[1] = deq_pair(w << 2, s2, c2);   // elements 2, 3 (bits 4-7, 20-23)
-  o[2] = deq_pair(w >> 2, s2, c2);   // elements 4, 5 (bits 8-11, 24-27)
-  o[3] = deq_pair(w >> 6, s2, c2);   // elements 6, 7 (bits 12-15, 28-31)
+  o[0] = deq_pair(w << 6, s2, c2);   // elements 0, 4 (bits 0-3, 16-19)
+  o[1] = deq_pair(w << 2, s2, c2);   // elements 1, 5 (bits 4-7, 20-23)
+  o[2] = deq_pair(w >> 2, s2, c2);   // elements 2, 6 (bits 8-11, 24-27)
+  o[3] = deq_pair(w >> 6, s2, c2);   // elements 3, 7 (bits 12-15, 28-31)
 }
 
 // s'' = s * 2^(e-6) and c = -1536 s'' as fp16 pairs
