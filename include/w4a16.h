@@ -105,9 +105,9 @@ w4_status w4_repack(const uint16_t* w, int64_t rows, int64_t K, uint32_t* codes,
  * element within a factor 2^27 of its row's largest), and every tensor-core product is exact;
  * the float32 sums and the final rounding are inexact.
  * Two kernels serve the call: for M < 64 (or N % 128 != 0, or K > 4096, or K % 64 != 0) a
- * weight-streaming kernel (workspace: M * ceil(K/256) * 656 bytes of prepared rows -- fp16
- * values, the row multiplier and per-group bias corrections -- and split-K partials), otherwise the
- * tensor-core kernel (workspace: M * K * 2 bytes and 4 per row, each rounded up to 256, plus one
+ * weight-streaming kernel (workspace: the prepared rows -- fp16 values, row multipliers and
+ * per-group bias corrections, in records of 8 or 16 rows per 512- or 256-k stage, about
+ * ceil(M/16) * ceil(K/256) * 10.3 KB -- and split-K partials), otherwise the tensor-core kernel (workspace: M * K * 2 bytes and 4 per row, each rounded up to 256, plus one
  * byte per weight row).  In the streaming kernel each
  * group's sum also carries a float32 rounding of a bias term that its correction cancels: about
  * 2^-13 of the group's mean |x| times 32 per group, far below the bf16 output rounding.
@@ -157,8 +157,10 @@ w4_status moe_route_permute(const float* logits, int32_t T, int32_t E, int32_t k
  *                   The tensor-core kernel (rows >= 32 * E, K <= 4096, K % 64 == 0, N % 128 == 0
  *                   or (N/2) % 64 == 0 with W4_EPI_GELU_GATE) needs rows * K * 2 bytes and 4
  *                   per row (each rounded up to 256) plus E * N bytes (a power-of-two exponent per
- *                   weight row); the weight-streaming kernel rows * ceil(K/256) * 656 bytes (fp16
- *                   values, the row multiplier and per-group bias corrections).
+ *                   weight row); the weight-streaming kernel one record per token block of 8
+ *                   or 16 rows of an expert and per 512- or 256-k stage (about 10 KB: fp16
+ *                   values, row multipliers and per-group bias corrections), for at most
+ *                   min(rows, rows / 8 + E) blocks, plus split-K partials for a few rows.
  *   dev_status      one int32 device word or NULL: set to a w4_status code if the device finds a
  *                   problem (offsets out of range: W4_ERR_INVALID_ARG; a pair naming a row past
  *                   the end of `a`: W4_ERR_INVALID_ARG, that row read as row 0); left unchanged

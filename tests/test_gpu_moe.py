@@ -135,7 +135,10 @@ def test_moe_small_batch_split_k(T):
     rows already fill more than half of the pipelines and take the unsplit path."""
     case = synth.moe_case(T, 128, 8, 2816, 704, seed=90 + T)
     rows = T * 8
-    prepared = 656 * (2816 // 256) * rows
+    # prepared records: one per (8-row token block, 512-k stage) of 8 x 1088 bytes of fp16 rows,
+    # 16 x 4 quads of 16 bytes and 8 multipliers; at most min(rows, rows // 8 + 128) blocks
+    blocks = min(rows, rows // 8 + min(128, rows))
+    prepared = blocks * ((2816 // 32 + 15) // 16) * (8 * 1088 + 16 * 4 * 16 + 8 * 4)
     ws = api.w4_workspace_bytes(_lib.W4_OP_GMM, rows, 2 * 704, 2816, 128, 8)
     if T == 1:
         assert ws > prepared + 3 * 4 * rows * 1408

@@ -39,9 +39,9 @@ def test_noalloc_matches_workspace_entry_point(M):
 
 
 def test_noalloc_splits_rows_that_do_not_fit_its_scratch():
-    """63 rows against K = 65536: the prepared activation rows alone (656 bytes per 256 k per
-    row) exceed the 8 MiB array, so the call runs the rows in chunks; the result must match the
-    regular entry point."""
+    """63 rows against K = 65536: the prepared activation rows alone (fp16 values, corrections
+    and multipliers of every 16-row block) exceed the 8 MiB array, so the call runs the rows in
+    chunks; the result must match the regular entry point."""
     lib = _lib.load()
     M, N, K = 63, 256, 65536
     need = api.w4_workspace_bytes(_lib.W4_OP_LINEAR, M, N, K, 1, 1)
