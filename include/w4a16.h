@@ -185,6 +185,23 @@ w4_status moe_combine(const uint16_t* o, const float* topk_w, const int32_t* pai
                       int32_t T, int32_t k, int32_t H, uint16_t* y, void* stream);
 
 /*
+ * moe_rms_chain -- the input of the next layer of a stack of MoE layers from this layer's output:
+ *   x_next[t, h] = bf16(y[t, h] / sqrt(mean_h y[t, h]^2 + eps)), rounded to nearest even.
+ * (No counterpart on the pages, which give no blocks between the MoE layers of a model; this is
+ * the plainest chaining that keeps a stack of gated expert MLPs -- quadratic in their input --
+ * bounded: a root-mean-square normalisation without a learned weight, eps = 1e-6 in this
+ * library's stack.)
+ *
+ *   y       [T, H] bf16 (input).    x_next  [T, H] bf16 (output; may not alias y).
+ *   T >= 0, H % 8 == 0, eps >= 0.  Both pointers 16-byte aligned.
+ * The sum of squares is float32 in a fixed order; the root and the division are correctly
+ * rounded float32, so an element can differ from the float64 definition by one bf16 unit where
+ * the quotient sits within float32 rounding of a bf16 midpoint.
+ */
+w4_status moe_rms_chain(const uint16_t* y, int64_t T, int32_t H, float eps, uint16_t* x_next,
+                        void* stream);
+
+/*
  * w4a16_linear_noalloc -- w4a16_linear for callers that cannot allocate device memory.
  * (No counterpart on the pages: an interface addition of this library.)
  *

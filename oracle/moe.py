@@ -20,7 +20,11 @@ not on the pages):
     ``pair_pos`` the inverse permutation;
   * the gate/up weight has 2I rows: rows 0..I-1 are the gate, rows I..2I-1 the up projection;
     h = gelu_tanh(gate) * up with gelu_tanh(z) = z/2 * (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3)));
-  * combine: y[t] = sum over slots j = 0..k-1 of w[t, j] * o[pair_pos[t*k + j]].
+  * combine: y[t] = sum over slots j = 0..k-1 of w[t, j] * o[pair_pos[t*k + j]];
+  * chaining of stacked layers (the pages give no blocks between the MoE layers, and the gated
+    expert MLP is quadratic in its input, so plain chaining grows without bound): the next
+    layer's input is the output divided by its root mean square, with no learned weight,
+    x_next = bf16(y / sqrt(mean(y^2) + eps)), eps = 1e-6.
 """
 from __future__ import annotations
 
@@ -164,3 +168,14 @@ def moe_layer(x_bits, logits, gu_codes, gu_scales, dn_codes, dn_scales, k: int,
             acc = acc + rt.topk_w[tokens, j:j + 1] * o[pp[tokens, j]]
         y[tokens] = acc
     return LayerResult(y=y, h=h, o=o, routing=rt)
+
+
+RMS_EPS = 1e-6
+
+
+def rms_chain(y_bits, eps: float = RMS_EPS) -> np.ndarray:
+    """Next layer's input from a layer's output: bf16(y / sqrt(mean over the row of y^2 + eps)),
+    per row, float64 then rounded to nearest even (bf16 bit patterns in and out)."""
+    y = bf16.to_f64(np.asarray(y_bits, dtype=np.uint16))
+    r = np.sqrt(np.mean(y * y, axis=-1, keepdims=True) + eps)
+    return bf16.from_f64(y / r)

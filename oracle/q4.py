@@ -51,16 +51,17 @@ def nibble_shift(j: int) -> int:
 
 
 def pack(q) -> np.ndarray:
-    """int codes [R, K] in -8..7 -> uint32 words [R, K/8] in the layout described above."""
-    q = np.asarray(q, dtype=np.int64)
+    """int codes [R, K] in -8..7 -> uint32 words [R, K/8] in the layout described above.
+
+    Nibble j of a word at bits 4j means, in bytes: byte b of the word (bits 8b..8b+7) holds
+    elements 2b (low nibble) and 2b + 1 (high nibble), and the word is read little-endian."""
+    q = np.asarray(q)
     R, K = q.shape
     assert K % 8 == 0
     assert q.min(initial=0) >= QMIN and q.max(initial=0) <= QMAX
-    u = (q + 8).astype(np.uint64).reshape(R, K // 8, 8)
-    word = np.zeros((R, K // 8), dtype=np.uint64)
-    for j in range(8):
-        word |= u[:, :, j] << np.uint64(nibble_shift(j))
-    return word.astype(np.uint32)
+    u = (q.astype(np.int16) + 8).astype(np.uint8).reshape(R, K // 2, 2)
+    byte = u[:, :, 0] | (u[:, :, 1] << np.uint8(4))
+    return np.ascontiguousarray(byte).view("<u4").reshape(R, K // 8).astype(np.uint32)
 
 
 def unpack(codes) -> np.ndarray:

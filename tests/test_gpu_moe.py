@@ -162,3 +162,55 @@ def test_moe_prefill_layer_sampled_tokens():
     layer, y, ref = _layer(case, tokens)
     assert np.array_equal(layer.rt.expert_offsets.cpu().numpy(), rt.expert_offsets)
     assert_rows_close(host_f64(y)[tokens], ref.y[tokens])
+
+
+def test_moe_prefill_layer_every_row():
+    """The prefill layer (8192 tokens, 128 Zipf(1.1)-skewed experts: hot experts with thousands
+    of rows, cold ones with a few, ragged last blocks) through the tensor-core kernel, checked on
+    every routed row: all 65,536 rows of h against the oracle's grouped GEMM with the GELU gate,
+    and all 65,536 rows of o against the oracle's down GEMM fed the device's own h (expert by
+    expert, so that only one chunk of float64 rows is held at a time)."""
+    case = synth.case_moe_prefill()
+    ref_rt = moe.route(case.logits, case.k)
+    dev = torch.device("cuda")
+    layer = api.MoELayer(dev_u32(case.gu_codes), dev_bf16(case.gu_scales), dev_u32(case.dn_codes),
+                         dev_bf16(case.dn_scales), case.T, case.k)
+    layer(dev_bf16(case.x), dev_f32(case.logits))
+    torch.cuda.synchronize()
+    assert np.array_equal(layer.rt.expert_offsets.cpu().numpy(), ref_rt.expert_offsets)
+    assert np.array_equal(layer.rt.sorted_pair.cpu().numpy(), ref_rt.sorted_pair)
+    counts = np.diff(ref_rt.expert_offsets)
+    assert counts.max() > 1000 and counts[counts > 0].min() < 10
+    h_ref = moe.gmm(case.x, ref_rt.sorted_pair, case.k, case.gu_codes, case.gu_scales,
+                    ref_rt.expert_offsets, moe.EPI_GELU_GATE)
+    assert_rows_close(host_f64(layer.h), h_ref, what="h")
+    del h_ref
+    h_bits = layer.h.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    o_dev = host_f64(layer.o)
+    off = ref_rt.expert_offsets.astype(np.int64)
+    e0 = 0
+    while e0 < case.E:
+        e1 = e0 + 1
+        while e1 < case.E and off[e1 + 1] - off[e0] <= 8192:
+            e1 += 1
+        r0, r1 = int(off[e0]), int(off[e1])
+        if r1 > r0:
+            o_ref = moe.gmm(h_bits[r0:r1], None, 1, case.dn_codes[e0:e1], case.dn_scales[e0:e1],
+                            off[e0:e1 + 1] - r0, moe.EPI_NONE)
+            assert_rows_close(o_dev[r0:r1], o_ref, what=f"o (experts {e0}..{e1 - 1})")
+        e0 = e1
+
+
+@pytest.mark.parametrize("T,H", [(1, 2816), (37, 2816), (256, 2816), (5, 8), (3, 4104)])
+def test_rms_chain_matches_oracle(T, H):
+    """moe_rms_chain against oracle.moe.rms_chain: every element within one bf16 unit (float32
+    sum of squares and quotient on the device, float64 in the oracle) and at least 99.9% of them
+    bit-identical."""
+    y = synth.bf16_normal((T, H), 0, 900 + T)
+    y = bf16.from_f64(bf16.to_f64(y) * (1 + np.arange(T)[:, None]))     # rows of different scale
+    x = api.moe_rms_chain(dev_bf16(y))
+    torch.cuda.synchronize()
+    got = x.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    ref = moe.rms_chain(y)
+    assert np.all(np.abs(got.astype(np.int32) - ref.astype(np.int32)) <= 1)
+    assert np.mean(got == ref) >= 0.999

@@ -158,3 +158,27 @@ def test_zipf_bias_skews_expert_loads():
     lg = synth.router_logits(8192, 128, 0, 102, zipf_s=synth.ZIPF_S)
     rt = moe.route(lg, 8)
     assert rt.counts.max() > 1000 and rt.counts.min() < 10
+
+
+def test_rms_chain_worked_example():
+    """y = [3, 4]: mean(y^2) = 12.5, sqrt(12.5 + 1e-6) = 3.5355340..., so y / rms =
+    [0.8485281..., 1.1313708...].  In bf16 (8 significant bits): 0.8485 = 1.69706 * 2^-1 and
+    1.69706 * 128 = 217.22 -> 217 / 128 * 2^-1 = 0.84765625 (0x3F59); 1.13137 * 128 = 144.82 ->
+    145 / 128 = 1.1328125 (0x3F91)."""
+    y = bf16.from_f64(np.array([[3.0, 4.0]]))
+    assert list(moe.rms_chain(y)[0]) == [0x3F59, 0x3F91]
+
+
+def test_rms_chain_constant_rows_and_scale_invariance():
+    # a constant row c (|c| >> eps) becomes +-1 exactly
+    y = bf16.from_f64(np.array([[2.5] * 64, [-0.375] * 64]))
+    x = bf16.to_f64(moe.rms_chain(y))
+    assert np.all(x[0] == 1.0) and np.all(x[1] == -1.0)
+    # scaling a row by a power of two (exact in bf16) changes nothing while eps stays negligible
+    rng = np.random.default_rng(5)
+    y = bf16.from_f64(rng.normal(size=(8, 2816)))
+    y4 = bf16.from_f64(bf16.to_f64(y) * 4.0)
+    assert np.array_equal(moe.rms_chain(y), moe.rms_chain(y4))
+    # the output row has mean square 1 up to the bf16 rounding of each element
+    x = bf16.to_f64(moe.rms_chain(y))
+    assert np.all(np.abs(np.mean(x * x, axis=1) - 1.0) < 2 ** -8)

@@ -38,6 +38,7 @@ SIGNATURES = {
                              _P, _P]),
     "moe_combine": (_I32, [_P, _P, _P, _I32, _I32, _I32, _P, _P]),
     "w4a16_linear_noalloc": (_I32, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "moe_rms_chain": (_I32, [_P, _I64, _I32, C.c_float, _P, _P]),
     "w4_workspace_bytes": (_SZ, [_I32, _I64, _I64, _I64, _I32, _I32]),
     "w4_status_str": (C.c_char_p, [_I32]),
     "w4_last_cuda_error": (_I32, []),

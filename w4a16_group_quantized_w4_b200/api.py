@@ -206,6 +206,22 @@ def moe_combine(o, topk_w, pair_pos, y=None, stream=None):
     return y
 
 
+RMS_EPS = 1e-6
+
+
+def moe_rms_chain(y, x_next=None, eps: float = RMS_EPS, stream=None):
+    """x_next [T, H] = bf16(y / sqrt(mean over each row of y^2 + eps)): the input of the next
+    layer of a stack (bf16 in and out)."""
+    lib = _lib.load()
+    T, H = y.shape
+    dev = y.device
+    _need("y", y, torch.bfloat16, (T, H), dev)
+    x_next = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if x_next is None else x_next
+    _need("x_next", x_next, torch.bfloat16, (T, H), dev)
+    _lib.check("moe_rms_chain", lib.moe_rms_chain(_p(y), T, H, eps, _p(x_next), _s(stream)))
+    return x_next
+
+
 class MoELayer:
     """One mixture-of-experts layer on the device: the four entry points composed on one stream
     (route -> gate/up GEMM with the GELU gate -> down GEMM -> combine), with every buffer

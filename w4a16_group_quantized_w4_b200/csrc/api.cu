@@ -16,12 +16,15 @@ w4_status w4_launch_route(const float* logits, int T, int E, int k, int32_t* ids
                           size_t ws_bytes, cudaStream_t stream);
 w4_status w4_launch_combine(const uint16_t* o, const float* topk_w, const int32_t* pair_pos, int T,
                             int k, int H, uint16_t* y, cudaStream_t stream);
+w4_status w4_launch_rms_chain(const uint16_t* y, int64_t T, int H, float eps, uint16_t* x,
+                              cudaStream_t stream, int sm_count);
 size_t w4_stream_workspace_bytes(int64_t rows, int N, int K, int E, int epi, bool dense, int sm_count);
 w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int k_div,
                                 const uint32_t* codes, const uint16_t* scales,
                                 const int32_t* offsets, int E, int64_t rows, int N, int K, int epi,
                                 uint16_t* out, void* ws, size_t ws_bytes, int32_t* dev_status,
-                                cudaStream_t stream, int sm_count);
+                                cudaStream_t stream, int sm_count, uint64_t wait_ns = 0,
+                                int stall_after = -1);
 size_t w4_tc_workspace_bytes(int64_t rows, int K, int64_t wrows);
 bool w4_tm_supported(int N, int K, int epi);
 w4_status w4_launch_tm_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int k_div,
@@ -185,12 +188,43 @@ w4_status moe_w4a16_gmm(const uint16_t* a, const int32_t* a_row_of_pair, int32_t
                                       static_cast<cudaStream_t>(stream), current_sm_count()));
 }
 
+// Fault injection for the tests of the bounded waits (not part of the C ABI in w4a16.h): the
+// grouped GEMM on the weight-streaming kernel with every wait limited to wait_ns and the producer
+// warps stopping after stall_after stages, so that the compute warps' waits run out.  The kernel
+// then reports W4_ERR_TIMEOUT in dev_status and returns; nothing faults or hangs.
+w4_status w4_testing_stream_gmm_stall(const uint16_t* a, const int32_t* a_row_of_pair, int32_t k,
+                                      const uint32_t* codes, const uint16_t* scales,
+                                      const int32_t* expert_offsets, int32_t E, int64_t rows, int32_t N,
+                                      int32_t K, int32_t epilogue, uint16_t* out, void* workspace,
+                                      size_t workspace_bytes, int32_t* dev_status, void* stream,
+                                      uint64_t wait_ns, int32_t stall_after) {
+  if (E < 1 || E > 1024 || rows < 0 || N < 1 || K < 32 || K % 32 || !codes || !scales || !expert_offsets)
+    return W4_ERR_INVALID_ARG;
+  if (epilogue != W4_EPI_NONE && epilogue != W4_EPI_GELU_GATE) return W4_ERR_INVALID_ARG;
+  if (rows > 0 && (!a || !out)) return W4_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(scales, 4) || (a && !aligned(a, 16)) || (out && !aligned(out, 16)))
+    return W4_ERR_INVALID_ARG;
+  return finish(w4_launch_stream_gemm(a, a_row_of_pair, k, codes, scales, expert_offsets, E, rows, N,
+                                      K, epilogue, out, workspace, workspace_bytes, dev_status,
+                                      static_cast<cudaStream_t>(stream), current_sm_count(), wait_ns,
+                                      stall_after));
+}
+
 w4_status moe_combine(const uint16_t* o, const float* topk_w, const int32_t* pair_pos, int32_t T,
                       int32_t k, int32_t H, uint16_t* y, void* stream) {
   if (T < 0 || k < 1 || H < 8 || H % 8) return W4_ERR_INVALID_ARG;
   if (T > 0 && (!o || !topk_w || !pair_pos || !y)) return W4_ERR_INVALID_ARG;
   if ((o && !aligned(o, 16)) || (y && !aligned(y, 16))) return W4_ERR_INVALID_ARG;
   return finish(w4_launch_combine(o, topk_w, pair_pos, T, k, H, y, static_cast<cudaStream_t>(stream)));
+}
+
+w4_status moe_rms_chain(const uint16_t* y, int64_t T, int32_t H, float eps, uint16_t* x_next,
+                        void* stream) {
+  if (T < 0 || H < 8 || H % 8 || !(eps >= 0.f) || eps > 1e30f) return W4_ERR_INVALID_ARG;
+  if (T > 0 && (!y || !x_next)) return W4_ERR_INVALID_ARG;
+  if ((y && !aligned(y, 16)) || (x_next && !aligned(x_next, 16))) return W4_ERR_INVALID_ARG;
+  return finish(w4_launch_rms_chain(y, T, H, eps, x_next, static_cast<cudaStream_t>(stream),
+                                    current_sm_count()));
 }
 
 }  // extern "C"

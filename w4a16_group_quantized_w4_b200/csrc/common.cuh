@@ -88,13 +88,14 @@ __device__ __forceinline__ bool mbar_try_wait_nohint(uint64_t* bar, uint32_t par
 }
 
 // Bounded wait of the streaming kernel's rings (no suspend hint: a waiting warp resumes sooner
-// once the phase completes); returns false once kWaitLimitNs have passed.
-__device__ __forceinline__ bool mbar_wait_ring(uint64_t* bar, uint32_t parity) {
+// once the phase completes); returns false once limit_ns have passed.
+__device__ __forceinline__ bool mbar_wait_ring(uint64_t* bar, uint32_t parity,
+                                               uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait_nohint(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait_nohint(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 

@@ -60,7 +60,8 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
                                 const uint32_t* codes, const uint16_t* scales,
                                 const int32_t* offsets, int E, int64_t rows, int N, int K, int epi,
                                 uint16_t* out, void* ws, size_t ws_bytes, int32_t* dev_status,
-                                cudaStream_t stream, int sm_count);
+                                cudaStream_t stream, int sm_count, uint64_t wait_ns = 0,
+                                int stall_after = -1);
 
 extern "C" {
 

@@ -360,6 +360,49 @@ __global__ void __launch_bounds__(128) combine_kernel(const uint16_t* __restrict
   *reinterpret_cast<uint4*>(y + static_cast<int64_t>(t) * H + h8 * 8) = out;
 }
 
+// ------------------------------------------------------------------------------------------
+// chaining of stacked layers: x[t] = bf16(y[t] / sqrt(mean(y[t]^2) + eps)).  One warp per row:
+// the lanes' float32 partial sums of squares over 16-byte chunks, combined by a fixed xor tree
+// (deterministic), then every element divided by the correctly rounded root (IEEE sqrt and
+// division) and rounded to bf16 (nearest even).  The row is read twice (the second time from
+// L1 / L2).
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) rms_chain_kernel(const uint16_t* __restrict__ y, int64_t T, int H,
+                                                        float eps, uint16_t* __restrict__ x) {
+  const int lane = threadIdx.x & 31;
+  const int64_t wpb = blockDim.x >> 5;
+  const int nv = H >> 3;
+  pdl_trigger();
+  pdl_wait();
+  for (int64_t t = blockIdx.x * wpb + (threadIdx.x >> 5); t < T; t += gridDim.x * wpb) {
+    const uint4* row = reinterpret_cast<const uint4*>(y + t * H);
+    float ss = 0.f;
+    for (int i = lane; i < nv; i += 32) {
+      const uint4 v = __ldg(row + i);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float a = bf16_lo_to_f32(w[q]), b = bf16_hi_to_f32(w[q]);
+        ss = fmaf(a, a, ss);
+        ss = fmaf(b, b, ss);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float r = __fsqrt_rn(__fdiv_rn(ss, static_cast<float>(H)) + eps);
+    uint4* out = reinterpret_cast<uint4*>(x + t * H);
+    for (int i = lane; i < nv; i += 32) {
+      const uint4 v = __ldg(row + i);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t o4[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        o4[q] = pack_bf16x2(__fdiv_rn(bf16_lo_to_f32(w[q]), r), __fdiv_rn(bf16_hi_to_f32(w[q]), r));
+      out[i] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+    }
+  }
+}
+
 }  // namespace w4
 
 // ---------------------------------------------------------------------------------------------
@@ -427,4 +470,14 @@ w4_status w4_launch_combine(const uint16_t* o, const float* topk_w, const int32_
   else e = launch_pdl(w4::combine_kernel<32>, grid, dim3(threads), 0, stream, o, topk_w, pair_pos, T, k, H, y);
   if (e != cudaSuccess) return W4_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+w4_status w4_launch_rms_chain(const uint16_t* y, int64_t T, int H, float eps, uint16_t* x,
+                              cudaStream_t stream, int sm_count) {
+  if (T == 0) return W4_OK;
+  const int64_t blocks = (T + 7) / 8;
+  const int grid = static_cast<int>(blocks < 8LL * sm_count ? blocks : 8LL * sm_count);
+  if (launch_pdl(w4::rms_chain_kernel, dim3(grid), dim3(256), 0, stream, y, T, H, eps, x) != cudaSuccess)
+    return W4_ERR_CUDA;
+  return W4_OK;
 }

@@ -54,12 +54,7 @@
 
 namespace w4 {
 
-#ifndef W4_STREAM_GROUPS_PER_PASS
-#define W4_STREAM_GROUPS_PER_PASS 4           // groups dequantised into registers at a time (MT = 16)
-#endif
-
 constexpr int kMaxStages = 6;
-constexpr int kGP = W4_STREAM_GROUPS_PER_PASS;
 constexpr int kWarps = 8;                     // compute warps per pipeline
 constexpr int kPipes = 2;                     // pipelines per CTA (one CTA per SM)
 constexpr int kPipeWarps = kWarps + 1;        // + one producer warp
@@ -127,6 +122,8 @@ struct StreamArgs {
   int pf_all;               // prefetch every stage of the pipeline's units into L2 at the start
   Layout L;
   int32_t* dev_status;
+  uint64_t wait_ns;         // limit of every bounded wait
+  int stall_after;          // fault injection for tests: producers stop after this many stages (< 0: never)
 };
 
 struct Unit {
@@ -312,18 +309,31 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     int slot = 0;
     uint32_t phase = 0;        // phase of the empty barrier to wait for on the next lap
     bool first_lap = true;
+    int64_t issued = 0;        // stages issued so far
+    // Before an early exit: wait (bounded) until the copies of the last S stages issued have
+    // landed, so that no bulk copy still writes into this CTA's shared memory after it exits.
+    // Stage i used slot i % S and completes phase (i / S) of that slot's full barrier.
+    auto drain = [&]() {
+      for (int64_t i = issued > S ? issued - S : 0; i < issued; ++i)
+        mbar_wait_ring(&full[i % S], static_cast<uint32_t>((i / S) & 1), A.wait_ns);
+    };
     // claims the next ring slot (false: a wait timed out or the compute warps gave up)
     auto claim = [&]() -> bool {
       if (!first_lap) {
-        if (!mbar_wait_ring(&empty[slot], phase) || flags[0]) {
+        if (!mbar_wait_ring(&empty[slot], phase, A.wait_ns) || flags[0]) {
           set_status(A.dev_status, W4_ERR_TIMEOUT);
           flags[0] = 1;
+          drain();
           return false;
         }
       }
+      if (A.stall_after >= 0 && issued >= A.stall_after) {   // (tests: the consumers' waits run out)
+        drain();
+        return false;
+      }
       return true;
     };
-    auto advance = [&]() { if (++slot == S) { slot = 0; if (!first_lap) phase ^= 1u; first_lap = false; } };
+    auto advance = [&]() { ++issued; if (++slot == S) { slot = 0; if (!first_lap) phase ^= 1u; first_lap = false; } };
     if (A.pf_all) {
       // weights that fit in L2 several times over: ask for all of this pipeline's code and scale
       // tiles now, so DRAM streams them at full rate while the ring fills from L2
@@ -452,7 +462,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
   auto epi_sync = [&]() -> bool {
     __syncwarp();
     if (lane == 0) mbar_arrive(epi_bar);
-    const bool ok = mbar_wait_ring(epi_bar, ephase);
+    const bool ok = mbar_wait_ring(epi_bar, ephase, A.wait_ns);
     ephase ^= 1u;
     if (!ok && lane == 0) { set_status(A.dev_status, W4_ERR_TIMEOUT); flags[0] = 1; }
     return ok;
@@ -470,7 +480,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     const uint32_t phase = cphase;
     if (++cslot == S) { cslot = 0; cphase ^= 1u; }
     // (a producer that gave up leaves its stage incomplete: this bounded wait then ends the warp)
-    if (!mbar_wait_ring(&full[slot], phase)) {
+    if (!mbar_wait_ring(&full[slot], phase, A.wait_ns)) {
       if (lane == 0) { set_status(A.dev_status, W4_ERR_TIMEOUT); flags[0] = 1; }
       return;
     }
@@ -1080,7 +1090,7 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
                                 const uint32_t* codes, const uint16_t* scales,
                                 const int32_t* offsets, int E, int64_t rows, int N, int K, int epi,
                                 uint16_t* out, void* ws, size_t ws_bytes, int32_t* dev_status,
-                                cudaStream_t stream, int sm_count) {
+                                cudaStream_t stream, int sm_count, uint64_t wait_ns, int stall_after) {
   const bool dense = (offsets == nullptr);
   StreamPlan p = plan_stream(rows, N, K, E, epi, dense, sm_count);
   w4::StreamArgs A{};
@@ -1089,6 +1099,8 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
   A.splits = p.splits; A.stages_per_split = p.stages_per_split; A.n_tiles = p.n_tiles;
   A.n_stages = p.n_stages;
   A.dev_status = dev_status;
+  A.wait_ns = wait_ns ? wait_ns : w4::kWaitLimitNs;
+  A.stall_after = stall_after;
   {
     // grouped calls whose experts' weights fit in half of L2 (a few decode tokens): prefetch
     // every stage at the start (a dense K = 4096 GEMV got slower with it: its ring's first loads

@@ -5,7 +5,8 @@ The whole-model form of the hot path: every layer's gate/up and down weights arr
 throughput", section "A repack, not a re-quantization"), are repacked on the device by
 `w4_repack` into int4 codes and bf16 scales, and decode steps then run the four entry points layer
 after layer ("The gap at 26B": 128 experts per layer, 8 active).  The pages give no blocks
-between the MoE layers, so each layer takes its own input rows and router logits.
+between the MoE layers; a chained step feeds each layer the previous layer's output divided by
+its root mean square (moe_rms_chain, no learned weight), with seeded router logits per layer.
 
 Layouts (layer-major, so layer l's weights are contiguous slices):
   gate/up codes [L, E, 2I, H/8] int32, scales [L, E, 2I, H/32] bf16
@@ -73,10 +74,29 @@ class MoEStack:
         return self._layers[key]
 
     def step(self, xs, logits, stream=None):
-        """One decode step through every layer: xs[l] bf16 [T, H], logits[l] f32 [T, E] -> the
-        list of layer outputs y_l bf16 [T, H] (each layer's own buffer)."""
+        """One decode step through every layer with independent inputs: xs[l] bf16 [T, H],
+        logits[l] f32 [T, E] -> the list of layer outputs y_l bf16 [T, H] (each layer's own
+        buffer)."""
         T = xs[0].shape[0]
         return [self.layer(l, T)(xs[l], logits[l], stream=stream) for l in range(self.L)]
+
+    def chained_step(self, x0, logits, stream=None):
+        """One decode step through the chained stack: layer 0 takes x0 bf16 [T, H]; layer l + 1
+        takes moe_rms_chain(y_l).  Returns (the inputs x_l, the outputs y_l), device buffers
+        owned by the stack (overwritten by the next chained step of the same T)."""
+        T = x0.shape[0]
+        key = ("chain", T)
+        if key not in self._layers:
+            self._layers[key] = [torch.empty((T, self.H), dtype=torch.bfloat16, device=x0.device)
+                                 for _ in range(self.L - 1)]
+        xb = self._layers[key]
+        xs, ys = [x0], []
+        for l in range(self.L):
+            y = self.layer(l, T)(xs[l], logits[l], stream=stream)
+            ys.append(y)
+            if l + 1 < self.L:
+                xs.append(api.moe_rms_chain(y, x_next=xb[l], stream=stream))
+        return xs, ys
 
     def expert_bytes(self) -> int:
         """Packed bytes of one expert (gate/up + down codes and scales)."""
