@@ -296,6 +296,20 @@ def native(args, world, rank, local):
     ms_per_step = ms / args.steps
     value = job_throughput(T * args.steps, world, ms)
 
+    # distribution of the step time: 100 graph replays, each between its own events
+    dist = []
+    with torch.cuda.stream(stream):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(100)]
+        for a, b in evs:
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+    stream.synchronize()
+    dist = sorted(a.elapsed_time(b) / spg for a, b in evs)
+    step_dist = {"n": len(dist), "unit": "ms per step", "median": round(float(np.median(dist)), 5),
+                 "p10": round(float(np.percentile(dist, 10)), 5), "p90": round(float(np.percentile(dist, 90)), 5),
+                 "how": f"100 replays of the {spg}-step graph, each between its own CUDA events, divided by {spg}"}
+
     # ---------------- per-kernel durations of the grouped GEMM (same launches) ----------------
     # Each GEMM call (its preparation pass included) replayed from a CUDA graph, alternating the
     # two weight copies, between CUDA events on the launch stream: the launch conditions of the
@@ -424,6 +438,7 @@ def native(args, world, rank, local):
                 "d2h_bytes_per_step": int(T * H * 2),
                 "how": f"public API (MoELayer) per step: pinned H2D of x and logits, 4 calls ({kernels} kernels), D2H of y"},
         "gpu_launches": kernels * args.steps,
+        "step_time_distribution": step_dist,
         "roofline": roofline,
         "cpu_baseline": cpu_base,
         "secondary": secondary,
@@ -459,9 +474,22 @@ def cpu_baseline(case):
                       case.k, tokens=tokens)
         done += len(tokens)
     dt = time.perf_counter() - t0
+    # the same oracle on one host thread, on the first chunk only
+    one = None
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            t1 = time.perf_counter()
+            moe.moe_layer(case.x, case.logits, case.gu_codes, case.gu_scales, case.dn_codes, case.dn_scales,
+                          case.k, tokens=np.arange(0, min(chunk, case.T)))
+            one = min(chunk, case.T) / (time.perf_counter() - t1)
+    except Exception:
+        pass
     return {"value": round(done / dt, 3), "unit": UNIT, "cores": int(threads), "kind": "oracle",
+            "value_1_thread": None if one is None else round(one, 3),
             "sample": f"{done} of {case.T} tokens of the same layer in chunks of {chunk} (routing of "
-                      f"all {case.T} each chunk); {dt:.1f} s of float64 numpy on the host"}
+                      f"all {case.T} each chunk); {dt:.1f} s of float64 numpy on the host; "
+                      f"value_1_thread: the first chunk with the BLAS pool limited to one thread"}
 
 
 def run_secondary(args, device, stream):
@@ -472,6 +500,29 @@ def run_secondary(args, device, stream):
     from w4a16_group_quantized_w4_b200 import api, synth
     out = {}
     hbm_peak, _, _, _ = peaks()
+    # the small dense linear (M = 4, K = 256, N = 256; launch-latency bound): graph-replayed calls
+    c1 = synth.case_dense_small()
+    xx, cc, ss = to_dev(c1.x, "bf16", device), to_dev(c1.codes, "u32", device), to_dev(c1.scales, "bf16", device)
+    yy = torch.empty((c1.M, c1.N), dtype=torch.bfloat16, device=device)
+    with torch.cuda.stream(stream):
+        for _ in range(5):
+            api.w4a16_linear(xx, cc, ss, y=yy)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(20):
+                api.w4a16_linear(xx, cc, ss, y=yy)
+        g.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(10):
+            g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    out["dense_small_M4_K256_N256"] = {"us_per_call": round(e0.elapsed_time(e1) * 1e3 / 200, 2),
+                                       "how": "200 calls in graphs of 20 (preparation pass + GEMM each)"}
+    del g
     # dense decode GEMV, K=4096, N=14336: 8 rotating weight copies (264 MB > 2x L2)
     base = synth.case_dense_gemv(16)
     nc = 8
@@ -537,7 +588,8 @@ def run_secondary(args, device, stream):
 
 def run_stack(device, stream, L=30, reps=3):
     """Repack + full expert stack: 30 layers x 128 experts of planted bf16 weights (generated on
-    the device), repacked, then decode steps through all 30 layers at 1, 32 and 256 tokens."""
+    the device), repacked, then decode steps through all 30 chained layers (layer l + 1 takes
+    moe_rms_chain of layer l's output) at 1, 32 and 256 tokens."""
     import torch
 
     from w4a16_group_quantized_w4_b200 import stack, synth, synth_device
@@ -564,14 +616,14 @@ def run_stack(device, stream, L=30, reps=3):
     del w_gu, w_dn, rep
     torch.cuda.empty_cache()
     for T in (1, 32, 256):
-        xs = [to_dev(synth.bf16_normal((T, H), 0, 600 + l), "bf16", device) for l in range(L)]
+        x0 = to_dev(synth.bf16_normal((T, H), 0, 600), "bf16", device)
         lgs = [to_dev(synth.router_logits(T, E, 0, 700 + l), "f32", device) for l in range(L)]
         with torch.cuda.stream(stream):
             for _ in range(2):
-                st.step(xs, lgs, stream=stream)
+                st.chained_step(x0, lgs, stream=stream)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                st.step(xs, lgs, stream=stream)
+                st.chained_step(x0, lgs, stream=stream)
             g.replay()
         stream.synchronize()
         hit = sum(int((torch.diff(st.layer(l, T).rt.expert_offsets) > 0).sum()) for l in range(L))
@@ -584,7 +636,7 @@ def run_stack(device, stream, L=30, reps=3):
             e1.record(stream)
         stream.synchronize()
         ms = e0.elapsed_time(e1) / n
-        byts = hit * st.expert_bytes() + L * T * H * 2 * 2
+        byts = hit * st.expert_bytes() + L * T * H * 2 * 2 + (L - 1) * T * H * 2 * 2   # + the chaining
         res[f"stack_decode_{L}_layers_T{T}"] = {"ms_per_step": round(ms, 3), "tokens/s": round(T / ms * 1e3, 1),
                                                "experts_hit": hit, "GB/s": round(byts / ms / 1e6, 1),
                                                "frac_hbm": round(byts / ms / 1e6 / hbm_peak, 3)}
