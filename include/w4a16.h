@@ -59,7 +59,9 @@ typedef enum {
 typedef enum {
   W4_OP_LINEAR = 1,
   W4_OP_ROUTE = 2,
-  W4_OP_GMM = 3
+  W4_OP_GMM = 3,
+  W4_OP_LINEAR_G = 4,       /* w4a16_linear_g (zero-points assumed present: an upper bound) */
+  W4_OP_GMM_G = 5           /* moe_w4a16_gmm_g (likewise) */
 } w4_op;
 
 /*
@@ -183,6 +185,33 @@ w4_status moe_w4a16_gmm(const uint16_t* a, const int32_t* a_row_of_pair, int32_t
  */
 w4_status moe_combine(const uint16_t* o, const float* topk_w, const int32_t* pair_pos,
                       int32_t T, int32_t k, int32_t H, uint16_t* y, void* stream);
+
+/*
+ * w4a16_linear_g, moe_w4a16_gmm_g -- the same linear and grouped GEMM on the weight-format
+ * variants: other group sizes along the input dimension and an asymmetric zero-point.
+ * ("What quantization really is", section "How the ruler works": a scale and an optional
+ * zero-point, asymmetric quantisation when values are not centred on zero, and group-wise
+ * granularity.  The page's formulas are lost in extraction; this is the standard uniform form.)
+ *
+ *   codes    as in layout L1, read as unsigned codes u in 0..15.
+ *   scales   [rows, K/group] bf16 (2-byte aligned): one scale per group of `group` elements.
+ *   zeros    [rows, K/group] uint8 zero-points z in 0..15, or NULL for the symmetric grid z = 8.
+ *   group    32, 64, 128, ... (32 times a power of two) dividing K.
+ *   Dequantised weight W = s * (u - z); group = 32 with zeros NULL is exactly the symmetric
+ *   format of w4a16_linear / moe_w4a16_gmm.  Every other argument, the workspace (sized with
+ *   W4_OP_LINEAR_G / W4_OP_GMM_G) and the accuracy statement are those of w4a16_linear /
+ *   moe_w4a16_gmm; both calls always take the weight-streaming kernel, scales and zero-points
+ *   loaded directly per stage (the zero-point's term (8 - z) * sum over the group of x enters
+ *   each group's MMA as part of its C operand, in float32).
+ */
+w4_status w4a16_linear_g(const uint16_t* x, const uint32_t* codes, const uint16_t* scales,
+                         const uint8_t* zeros, int32_t group, uint16_t* y, int64_t M, int64_t N,
+                         int64_t K, void* workspace, size_t workspace_bytes, void* stream);
+w4_status moe_w4a16_gmm_g(const uint16_t* a, const int32_t* a_row_of_pair, int32_t k,
+                          const uint32_t* codes, const uint16_t* scales, const uint8_t* zeros,
+                          int32_t group, const int32_t* expert_offsets, int32_t E, int64_t rows,
+                          int32_t N, int32_t K, int32_t epilogue, uint16_t* out, void* workspace,
+                          size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
  * moe_rms_chain -- the input of the next layer of a stack of MoE layers from this layer's output:

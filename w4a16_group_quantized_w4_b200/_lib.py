@@ -24,6 +24,8 @@ W4_EPI_GELU_GATE = 1
 W4_OP_LINEAR = 1
 W4_OP_ROUTE = 2
 W4_OP_GMM = 3
+W4_OP_LINEAR_G = 4
+W4_OP_GMM_G = 5
 
 # name -> (restype, argtypes), mirroring include/w4a16.h
 _P = C.c_void_p
@@ -39,6 +41,9 @@ SIGNATURES = {
     "moe_combine": (_I32, [_P, _P, _P, _I32, _I32, _I32, _P, _P]),
     "w4a16_linear_noalloc": (_I32, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "moe_rms_chain": (_I32, [_P, _I64, _I32, C.c_float, _P, _P]),
+    "w4a16_linear_g": (_I32, [_P, _P, _P, _P, _I32, _P, _I64, _I64, _I64, _P, _SZ, _P]),
+    "moe_w4a16_gmm_g": (_I32, [_P, _P, _I32, _P, _P, _P, _I32, _P, _I32, _I64, _I32, _I32, _I32, _P,
+                               _P, _SZ, _P, _P]),
     "w4_workspace_bytes": (_SZ, [_I32, _I64, _I64, _I64, _I32, _I32]),
     "w4_status_str": (C.c_char_p, [_I32]),
     "w4_last_cuda_error": (_I32, []),

@@ -103,6 +103,28 @@ def w4a16_linear(x, codes, scales, y=None, ws=None, stream=None):
     return y
 
 
+def w4a16_linear_g(x, codes, scales, group: int, zeros=None, y=None, ws=None, stream=None):
+    """The linear on the weight-format variants: scales [N, K/group] bf16, zeros [N, K/group]
+    uint8 zero-points (or None: z = 8); W = s * (u - z)."""
+    lib = _lib.load()
+    M, K = x.shape
+    N = codes.shape[0]
+    dev = x.device
+    _need("x", x, torch.bfloat16)
+    _need("codes", codes, torch.int32, (N, K // 8), dev)
+    _need("scales", scales, torch.bfloat16, (N, K // group), dev)
+    if zeros is not None:
+        _need("zeros", zeros, torch.uint8, (N, K // group), dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev) if y is None else y
+    _need("y", y, torch.bfloat16, (M, N), dev)
+    if ws is None:
+        ws = workspace(w4_workspace_bytes(_lib.W4_OP_LINEAR_G, M, N, K, 1, 1), dev)
+    _lib.check("w4a16_linear_g", lib.w4a16_linear_g(_p(x), _p(codes), _p(scales), _p(zeros), group, _p(y),
+                                                    M, N, K, _p(ws), 0 if ws is None else ws.numel(),
+                                                    _s(stream)))
+    return y
+
+
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -220,6 +242,39 @@ def moe_rms_chain(y, x_next=None, eps: float = RMS_EPS, stream=None):
     _need("x_next", x_next, torch.bfloat16, (T, H), dev)
     _lib.check("moe_rms_chain", lib.moe_rms_chain(_p(y), T, H, eps, _p(x_next), _s(stream)))
     return x_next
+
+
+def moe_w4a16_gmm_g(a, a_row_of_pair, k: int, codes, scales, expert_offsets, rows: int, group: int,
+                    zeros=None, epilogue: int = W4_EPI_NONE, out=None, ws=None, dev_status=None,
+                    stream=None):
+    """The grouped GEMM on the weight-format variants: scales [E, N, K/group], zeros
+    [E, N, K/group] uint8 or None."""
+    lib = _lib.load()
+    E, N, Kw = codes.shape
+    K = Kw * 8
+    dev = a.device
+    _need("a", a, torch.bfloat16)
+    if a.shape[1] != K:
+        raise ValueError("a: wrong number of columns")
+    if a_row_of_pair is not None:
+        _need("a_row_of_pair", a_row_of_pair, torch.int32, (rows,), dev)
+    _need("codes", codes, torch.int32, (E, N, K // 8), dev)
+    _need("scales", scales, torch.bfloat16, (E, N, K // group), dev)
+    if zeros is not None:
+        _need("zeros", zeros, torch.uint8, (E, N, K // group), dev)
+    _need("expert_offsets", expert_offsets, torch.int32, (E + 1,), dev)
+    n_out = N // 2 if epilogue == W4_EPI_GELU_GATE else N
+    out = torch.empty((rows, n_out), dtype=torch.bfloat16, device=dev) if out is None else out
+    _need("out", out, torch.bfloat16, (rows, n_out), dev)
+    if ws is None:
+        ws = workspace(w4_workspace_bytes(_lib.W4_OP_GMM_G, rows, N, K, E, k), dev)
+    if dev_status is not None:
+        _need("dev_status", dev_status, torch.int32, (1,), dev)
+    _lib.check("moe_w4a16_gmm_g", lib.moe_w4a16_gmm_g(
+        _p(a), _p(a_row_of_pair), k, _p(codes), _p(scales), _p(zeros), group, _p(expert_offsets), E,
+        rows, N, K, epilogue, _p(out), _p(ws), 0 if ws is None else ws.numel(), _p(dev_status),
+        _s(stream)))
+    return out
 
 
 class MoELayer:

@@ -18,13 +18,14 @@ w4_status w4_launch_combine(const uint16_t* o, const float* topk_w, const int32_
                             int k, int H, uint16_t* y, cudaStream_t stream);
 w4_status w4_launch_rms_chain(const uint16_t* y, int64_t T, int H, float eps, uint16_t* x,
                               cudaStream_t stream, int sm_count);
-size_t w4_stream_workspace_bytes(int64_t rows, int N, int K, int E, int epi, bool dense, int sm_count);
+size_t w4_stream_workspace_bytes(int64_t rows, int N, int K, int E, int epi, bool dense, int sm_count,
+                                 bool zp = false);
 w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int k_div,
                                 const uint32_t* codes, const uint16_t* scales,
                                 const int32_t* offsets, int E, int64_t rows, int N, int K, int epi,
                                 uint16_t* out, void* ws, size_t ws_bytes, int32_t* dev_status,
                                 cudaStream_t stream, int sm_count, uint64_t wait_ns = 0,
-                                int stall_after = -1);
+                                int stall_after = -1, const uint8_t* zeros = nullptr, int group = 32);
 size_t w4_tc_workspace_bytes(int64_t rows, int K, int64_t wrows);
 bool w4_tm_supported(int N, int K, int epi);
 w4_status w4_launch_tm_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int k_div,
@@ -115,6 +116,22 @@ size_t w4_workspace_bytes(int32_t op, int64_t M_or_T, int64_t N, int64_t K, int3
       }
       return need;
     }
+    case W4_OP_LINEAR_G:
+    case W4_OP_GMM_G:
+      // the variants always take the weight-streaming kernel; sized for zero-points (the larger)
+      if (N <= 0 || K < 32 || K % 32 || E < 1 || N > (1LL << 30) || K > (1LL << 30)) return 0;
+      if (op == W4_OP_LINEAR_G)
+        return w4_stream_workspace_bytes(M_or_T, static_cast<int>(N), static_cast<int>(K), 1, W4_EPI_NONE,
+                                         true, current_sm_count(), true);
+      {
+        size_t need = 0;
+        for (int epi : {W4_EPI_NONE, W4_EPI_GELU_GATE}) {
+          const size_t b = w4_stream_workspace_bytes(M_or_T, static_cast<int>(N), static_cast<int>(K), E, epi,
+                                                     false, current_sm_count(), true);
+          if (b > need) need = b;
+        }
+        return need;
+      }
     default:
       return 0;
   }
@@ -208,6 +225,50 @@ w4_status w4_testing_stream_gmm_stall(const uint16_t* a, const int32_t* a_row_of
                                       K, epilogue, out, workspace, workspace_bytes, dev_status,
                                       static_cast<cudaStream_t>(stream), current_sm_count(), wait_ns,
                                       stall_after));
+}
+
+static bool group_ok(int64_t group, int64_t K) {
+  if (group < 32 || group > K || K % group) return false;
+  int64_t g = group / 32;
+  return group % 32 == 0 && (g & (g - 1)) == 0;
+}
+
+w4_status w4a16_linear_g(const uint16_t* x, const uint32_t* codes, const uint16_t* scales,
+                         const uint8_t* zeros, int32_t group, uint16_t* y, int64_t M, int64_t N, int64_t K,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (M < 0 || N < 1 || K < 32 || K % 32 || N > (1LL << 30) || K > (1LL << 30)) return W4_ERR_INVALID_ARG;
+  if (!group_ok(group, K)) return W4_ERR_INVALID_ARG;
+  if (M > 0 && (!x || !y)) return W4_ERR_INVALID_ARG;
+  if (!codes || !scales) return W4_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(scales, 2) || (x && !aligned(x, 16)) || (y && !aligned(y, 16)))
+    return W4_ERR_INVALID_ARG;
+  if (workspace && !aligned(workspace, 16)) return W4_ERR_INVALID_ARG;
+  if (M * N > (1LL << 40)) return W4_ERR_UNSUPPORTED;
+  return finish(w4_launch_stream_gemm(x, nullptr, 1, codes, scales, nullptr, 1, M, static_cast<int>(N),
+                                      static_cast<int>(K), W4_EPI_NONE, y, workspace, workspace_bytes,
+                                      nullptr, static_cast<cudaStream_t>(stream), current_sm_count(), 0, -1,
+                                      zeros, group));
+}
+
+w4_status moe_w4a16_gmm_g(const uint16_t* a, const int32_t* a_row_of_pair, int32_t k,
+                          const uint32_t* codes, const uint16_t* scales, const uint8_t* zeros,
+                          int32_t group, const int32_t* expert_offsets, int32_t E, int64_t rows,
+                          int32_t N, int32_t K, int32_t epilogue, uint16_t* out, void* workspace,
+                          size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  if (E < 1 || E > 1024 || rows < 0 || N < 1 || K < 32 || K % 32) return W4_ERR_INVALID_ARG;
+  if (!group_ok(group, K)) return W4_ERR_INVALID_ARG;
+  if (epilogue != W4_EPI_NONE && epilogue != W4_EPI_GELU_GATE) return W4_ERR_INVALID_ARG;
+  if (epilogue == W4_EPI_GELU_GATE && (N % 2)) return W4_ERR_INVALID_ARG;
+  if (a_row_of_pair && k < 1) return W4_ERR_INVALID_ARG;
+  if (!codes || !scales || !expert_offsets) return W4_ERR_INVALID_ARG;
+  if (rows > 0 && (!a || !out)) return W4_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(scales, 2) || (a && !aligned(a, 16)) || (out && !aligned(out, 16)))
+    return W4_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(E) * N > (1LL << 31) - 1 || rows > (1LL << 31) - 1) return W4_ERR_UNSUPPORTED;
+  return finish(w4_launch_stream_gemm(a, a_row_of_pair, k, codes, scales, expert_offsets, E, rows, N, K,
+                                      epilogue, out, workspace, workspace_bytes, dev_status,
+                                      static_cast<cudaStream_t>(stream), current_sm_count(), 0, -1, zeros,
+                                      group));
 }
 
 w4_status moe_combine(const uint16_t* o, const float* topk_w, const int32_t* pair_pos, int32_t T,

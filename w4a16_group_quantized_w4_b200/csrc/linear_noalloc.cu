@@ -55,13 +55,14 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 // from stream_gemm.cu / api.cu (w4_record_status: records the CUDA error behind a W4_ERR_CUDA
 // for w4_last_cuda_error, as every other entry point does)
 w4_status w4_record_status(w4_status s);
-size_t w4_stream_workspace_bytes(int64_t rows, int N, int K, int E, int epi, bool dense, int sm_count);
+size_t w4_stream_workspace_bytes(int64_t rows, int N, int K, int E, int epi, bool dense, int sm_count,
+                                 bool zp = false);
 w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int k_div,
                                 const uint32_t* codes, const uint16_t* scales,
                                 const int32_t* offsets, int E, int64_t rows, int N, int K, int epi,
                                 uint16_t* out, void* ws, size_t ws_bytes, int32_t* dev_status,
                                 cudaStream_t stream, int sm_count, uint64_t wait_ns = 0,
-                                int stall_after = -1);
+                                int stall_after = -1, const uint8_t* zeros = nullptr, int group = 32);
 
 extern "C" {
 

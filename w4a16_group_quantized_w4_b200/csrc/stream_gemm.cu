@@ -75,21 +75,26 @@ enum ScaleMode { kScaleLdg = 0, kScaleBlock = 1, kScaleTma = 2 };
 //   [MT rows x rec_xp bytes of x' (GS * 64 bytes, padded so that consecutive rows sit 64 bytes
 //    apart in the shared-memory banks)]
 //   [quads: group-major, GS x MT/2 row pairs x 16 bytes {c(r), c(r+1), c(r), c(r+1)}]
-//   [MT row multipliers 2^-f (float)], padded to 16 bytes.
+//   [MT row multipliers 2^-f (float)], padded to 16 bytes
+//   [zero-point variant only: group-major, GS x MT/2 row pairs x 8 bytes {Sx(r), Sx(r+1)}, the
+//    sum over the group of the row's x' values], padded to 16 bytes.
 __host__ __device__ constexpr int rec_xp(int GS) { return GS * 64 + 64; }
 __host__ __device__ constexpr int rec_qoff(int MT, int GS) { return MT * rec_xp(GS); }
 __host__ __device__ constexpr int rec_moff(int MT, int GS) { return rec_qoff(MT, GS) + GS * (MT / 2) * 16; }
-__host__ __device__ constexpr int rec_bytes(int MT, int GS) { return (rec_moff(MT, GS) + MT * 4 + 15) & ~15; }
+__host__ __device__ constexpr int rec_soff(int MT, int GS) { return (rec_moff(MT, GS) + MT * 4 + 15) & ~15; }
+__host__ __device__ constexpr int rec_bytes(int MT, int GS, bool ZP = false) {
+  return ZP ? (rec_soff(MT, GS) + GS * (MT / 2) * 8 + 15) & ~15 : rec_soff(MT, GS);
+}
 
 // Shared-memory slot of one stage (offsets from the slot base, a multiple of 1024 bytes):
 //   codes: GS/8 column boxes x 2 row halves x 8 KB; then the prepared record; then the stage
 //   descriptor; then the scales.
 __host__ __device__ constexpr int slot_code_bytes(int GS) { return (GS / kBoxG) * 2 * kBoxBytes; }
 __host__ __device__ constexpr int slot_act_off(int GS) { return slot_code_bytes(GS); }
-__host__ __device__ constexpr int slot_desc_off(int MT, int GS) {
-  return slot_act_off(GS) + ((rec_bytes(MT, GS) + 127) & ~127);
+__host__ __device__ constexpr int slot_desc_off(int MT, int GS, bool ZP = false) {
+  return slot_act_off(GS) + ((rec_bytes(MT, GS, ZP) + 127) & ~127);
 }
-__host__ __device__ constexpr int slot_sc_off(int MT, int GS) { return slot_desc_off(MT, GS) + 128; }
+__host__ __device__ constexpr int slot_sc_off(int MT, int GS, bool ZP = false) { return slot_desc_off(MT, GS, ZP) + 128; }
 
 // Shared-memory layout of one launch (offsets from the 1024-byte aligned base): pipeline p's
 // ring at p * pipe_bytes, its split-K epilogue buffer, barriers and flags after the ring; then the
@@ -110,7 +115,9 @@ struct Layout {
 struct StreamArgs {
   const uint8_t* xw;        // prepared records: [token block][stage][rec_bytes]
   int n_stages;             // stages per row (ceil(K / (GS * 32)))
-  const uint16_t* scales;   // [E*N, kg]
+  const uint16_t* scales;   // [E*N, kgs]: one bf16 per group of 32 << gshift
+  const uint8_t* zeros;     // [E*N, kgs] zero-points 0..15 (zero-point variant) or null
+  int gshift, kgs;          // scale group = 32 << gshift elements; scales per row
   const int32_t* offsets;   // [E+1] or null (one expert with `rows` rows)
   int E, N, K, kg;
   int64_t rows;
@@ -218,14 +225,15 @@ __device__ __forceinline__ float scale_of(const uint32_t* w, int gi) {
   return __uint_as_float((gi & 1) ? (w[gi >> 1] & 0xFFFF0000u) : (w[gi >> 1] << 16));
 }
 
-template <int MT, int GS, bool GELU, int SCALE>
+template <int MT, int GS, bool GELU, int SCALE, bool ZP>
 __global__ void __launch_bounds__(kThreads, 1)
 stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
                    const __grid_constant__ CUtensorMap tmap_scales, StreamArgs A) {
   constexpr int kActOff = slot_act_off(GS);
-  constexpr int kDescOff = slot_desc_off(MT, GS);
-  constexpr int kScOff = slot_sc_off(MT, GS);
-  constexpr int kRec = rec_bytes(MT, GS);
+  constexpr int kDescOff = slot_desc_off(MT, GS, ZP);
+  constexpr int kScOff = slot_sc_off(MT, GS, ZP);
+  constexpr int kRec = rec_bytes(MT, GS, ZP);
+  constexpr int kSOff = rec_soff(MT, GS);
   constexpr int kXP = rec_xp(GS);
   constexpr int kQOff = rec_qoff(MT, GS);
   constexpr int kMOff = rec_moff(MT, GS);
@@ -499,8 +507,10 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     const int g0 = short_stage ? kp * (kGW / 2) : kp * kGW;   // this warp's first group
     const int sg0 = short_stage ? 0 : kp * kGW;                // first group of the scales loaded
     {
-      // scales of the thread's four rows for its kGW groups, two bf16 per word
+      // scales of the thread's four rows for its kGW groups, two bf16 per word; zero-points
+      // (variant), four bytes per word
       uint32_t sw[4][kGW / 2];
+      uint32_t zw[4][ZP ? kGW / 4 : 1];
       if (SCALE == kScaleTma) {
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
@@ -523,6 +533,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           for (int q = 0; q < kGW / 2; ++q) sw[r][q] = sg0 + 2 * q < gc ? p[q] : 0u;
         }
       } else {
+        // direct loads (also every other scale group size: group gi of 32 uses scale gi >> gshift)
         const int4 d1 = *reinterpret_cast<const int4*>(sp8 + kDescOff + 16);
         const int dnt = static_cast<int>(d0.z), de = d1.x;
 #pragma unroll
@@ -531,18 +542,36 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
 #pragma unroll
           for (int q = 0; q < kGW / 2; ++q) {
             const int ga = g + sg0 + 2 * q;
-            const uint32_t l0 = ga - g < gc ? ldg_u16(A.scales + grow * A.kg + ga) : 0;
-            const uint32_t l1 = ga + 1 - g < gc ? ldg_u16(A.scales + grow * A.kg + ga + 1) : 0;
+            const uint32_t l0 = ga - g < gc ? ldg_u16(A.scales + grow * A.kgs + (ga >> A.gshift)) : 0;
+            const uint32_t l1 = ga + 1 - g < gc ? ldg_u16(A.scales + grow * A.kgs + ((ga + 1) >> A.gshift)) : 0;
             sw[r][q] = l0 | (l1 << 16);
+          }
+          if (ZP) {
+#pragma unroll
+            for (int q = 0; q < kGW / 4; ++q) {
+              uint32_t word = 0;
+#pragma unroll
+              for (int b = 0; b < 4; ++b) {
+                const int ga = g + sg0 + 4 * q + b;
+                const uint32_t zv = ga - g < gc ? __ldg(A.zeros + grow * A.kgs + (ga >> A.gshift)) : 8u;
+                word |= zv << (8 * b);
+              }
+              zw[r][q] = word;
+            }
           }
         }
       }
       if (short_stage && kp == 1) {
         // this warp's groups are the second half of the scales loaded
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < 4; ++r) {
 #pragma unroll
           for (int q = 0; q < kGW / 4; ++q) sw[r][q] = sw[r][q + kGW / 4];
+          if (ZP) {
+#pragma unroll
+            for (int q = 0; q < kGW / 8; ++q) zw[r][q] = zw[r][q + kGW / 8];
+          }
+        }
       }
       // The warp's groups g0 + i, i = 0.. (compile-time): groups 8..15 of a full 16-group stage
       // sit in the second column box; four-group halves (a short stage, or GS = 8) are chunks
@@ -553,6 +582,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
                                                         : (sb + cbase) ^ static_cast<uint32_t>(kp << 6);
       const uint32_t xg = sb + kActOff + gid * kXP + tq * 16 + g0 * 64;
       const uint32_t qg = sb + kActOff + kQOff + tq * 16 + g0 * (MT / 2) * 16;   // row pair (2tq, 2tq + 1)
+      const uint32_t sg = sb + kActOff + kSOff + tq * 8 + g0 * (MT / 2) * 8;      // (zero-point variant)
       const int nblk = NB == 1 ? 1 : (mt + 7) >> 3;
       const int ngw = short_stage ? kGW / 2 : kGW;
 #pragma unroll
@@ -566,11 +596,26 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           if (b >= nblk) break;
           const uint4 xv = lds128(xg + b * 8 * kXP + i * 64);
           const uint4 cq = lds128(qg + b * 4 * 16 + i * (MT / 2) * 16);
-          const float c[4] = {__uint_as_float(cq.x), __uint_as_float(cq.y), __uint_as_float(cq.z),
-                              __uint_as_float(cq.w)};
+          float c[4] = {__uint_as_float(cq.x), __uint_as_float(cq.y), __uint_as_float(cq.z),
+                        __uint_as_float(cq.w)};
+          float c1[4] = {c[0], c[1], c[2], c[3]};
+          if (ZP) {
+            // sum (u - z) x' = sum (u - 8) x' + (8 - z) Sx: the zero-point enters the C operand
+            // per (row, token)
+            const uint2 sx = lds64(sg + b * 4 * 8 + i * (MT / 2) * 8);
+            const float sx0 = __uint_as_float(sx.x), sx1 = __uint_as_float(sx.y);
+            float dz[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+              dz[r] = static_cast<float>(8 - static_cast<int>((zw[r][i >> 2] >> (8 * (i & 3))) & 0xFFu));
+            c[0] = fmaf(dz[0], sx0, c[0]); c[1] = fmaf(dz[0], sx1, c[1]);
+            c[2] = fmaf(dz[1], sx0, c[2]); c[3] = fmaf(dz[1], sx1, c[3]);
+            c1[0] = fmaf(dz[2], sx0, c1[0]); c1[1] = fmaf(dz[2], sx1, c1[1]);
+            c1[2] = fmaf(dz[3], sx0, c1[2]); c1[3] = fmaf(dz[3], sx1, c1[3]);
+          }
           float p0[4], p1[4];
           mma_nib(p0, w00, w01, xv.x, xv.y, c, e1024);
-          mma_nib(p1, w10, w11, xv.x, xv.y, c, e1024);
+          mma_nib(p1, w10, w11, xv.x, xv.y, c1, e1024);
           mma_nib(p0, w00 >> 8, w01 >> 8, xv.z, xv.w, p0, e1024);
           mma_nib(p1, w10 >> 8, w11 >> 8, xv.z, xv.w, p1, e1024);
           const float s0 = scale_of(sw[0], i), s1 = scale_of(sw[1], i);
@@ -773,17 +818,19 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
 // over its 4 lanes (from the stored fp16 values), into components (slot & 1) and (slot & 1) + 2
 // of the row pair's quad.  Elements past K are written as zero, up to the end of the last stage.
 // Every stage's record also carries the row's multiplier 2^-f, so that a unit's epilogue finds
-// it next to its last stage.
-template <int MT, int GS>
+// it next to its last stage.  The zero-point variant also stores each group's sum of the row's x'
+// values, Sx = (first + third pairs) + 16 (second + fourth pairs), into the row pair's Sx slot.
+template <int MT, int GS, bool ZP>
 __global__ void __launch_bounds__(256)
 stream_prep_kernel(const uint16_t* __restrict__ a, const int32_t* __restrict__ a_row_of_pair, int k_div,
                    int64_t a_rows, int64_t rows, int K, const int32_t* __restrict__ offsets, int E,
                    uint8_t* __restrict__ xw, int n_stages, int64_t n_blocks, int32_t* __restrict__ counters,
                    int n_counters, int32_t* dev_status) {
-  constexpr int kRec = rec_bytes(MT, GS);
+  constexpr int kRec = rec_bytes(MT, GS, ZP);
   constexpr int kXP = rec_xp(GS);
   constexpr int kQOff = rec_qoff(MT, GS);
   constexpr int kMOff = rec_moff(MT, GS);
+  constexpr int kSOff = rec_soff(MT, GS);
   constexpr int kBPS = GS / kBoxG;               // 256-k blocks per stage
   extern __shared__ int prep_smem[];
   int* offs = prep_smem;                          // [E + 1]
@@ -894,17 +941,24 @@ stream_prep_kernel(const uint16_t* __restrict__ a, const int32_t* __restrict__ a
         const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h[1]));
         const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&h[2]));
         const float2 f3 = __half22float2(*reinterpret_cast<const __half2*>(&h[3]));
-        float part = 1032.f * ((f0.x + f0.y) + (f2.x + f2.y)) + 1152.f * ((f1.x + f1.y) + (f3.x + f3.y));
+        const float sa = (f0.x + f0.y) + (f2.x + f2.y), sb = (f1.x + f1.y) + (f3.x + f3.y);
+        float part = 1032.f * sa + 1152.f * sb;
+        float sxp = ZP ? sa + 16.f * sb : 0.f;
         uint8_t* rec = rec0 + static_cast<int64_t>(j / kBPS) * kRec;
         const int sub = j % kBPS;                 // 256-k block within the stage
         *reinterpret_cast<uint4*>(rec + slot * kXP + (sub * 32 + lane) * 16) = make_uint4(h[0], h[1], h[2], h[3]);
         part += __shfl_xor_sync(0xffffffffu, part, 1);
         part += __shfl_xor_sync(0xffffffffu, part, 2);
+        if (ZP) {
+          sxp += __shfl_xor_sync(0xffffffffu, sxp, 1);
+          sxp += __shfl_xor_sync(0xffffffffu, sxp, 2);
+        }
         if ((lane & 3) == 0) {
           const int gi = sub * kBoxG + (lane >> 2);
           float* q = reinterpret_cast<float*>(rec + kQOff + (gi * (MT / 2) + (slot >> 1)) * 16) + (slot & 1);
           q[0] = -part;
           q[2] = -part;
+          if (ZP) reinterpret_cast<float*>(rec + kSOff + (gi * (MT / 2) + (slot >> 1)) * 8)[slot & 1] = sxp;
         }
       }
     }
@@ -962,11 +1016,11 @@ static bool encode_scales_map(CUtensorMap* m, const uint16_t* scales, int64_t ro
 
 // Ring depth and offsets for one launch: each of the CTA's two pipelines gets half of the shared
 // memory left next to the unit table, with as many slots (up to kMaxStages) as fit.
-static w4::Layout make_layout(int MT, int GS, int scale_mode, int kg, int E, bool split) {
+static w4::Layout make_layout(int MT, int GS, int scale_mode, int kg, int E, bool split, bool zp) {
   w4::Layout L{};
   L.sc_bytes = scale_mode == w4::kScaleTma ? 2 * w4::kHalf * GS * 2
              : scale_mode == w4::kScaleBlock ? 2 * w4::kHalf * kg * 2 : 0;
-  L.slot_bytes = (w4::slot_sc_off(MT, GS) + L.sc_bytes + 1023) & ~1023;
+  L.slot_bytes = (w4::slot_sc_off(MT, GS, zp) + L.sc_bytes + 1023) & ~1023;
   const int table_bytes = (E + 1) * 12;
   const int ep_bytes = split ? MT * w4::kEpPitch * 4 : 0;
   const int red_bytes = 2 * 4 * (MT / 8) * 2 * 32 * 16;
@@ -1034,9 +1088,9 @@ static int64_t block_capacity(int64_t rows, int MT, int E, bool dense) {
   return std::min<int64_t>(rows, rows / MT + std::min<int64_t>(E, rows));
 }
 
-static size_t prep_bytes(const StreamPlan& p, int64_t rows, int E, bool dense) {
+static size_t prep_bytes(const StreamPlan& p, int64_t rows, int E, bool dense, bool zp) {
   return align256(static_cast<size_t>(block_capacity(rows, p.MT, E, dense)) * p.n_stages *
-                  w4::rec_bytes(p.MT, p.GS));
+                  w4::rec_bytes(p.MT, p.GS, zp));
 }
 
 // one arrival counter per (expert, token block, weight tile)
@@ -1044,58 +1098,69 @@ static size_t counters_bytes(const StreamPlan& p, int64_t rows, int E, bool dens
   return align256(static_cast<size_t>(block_capacity(rows, p.MT, E, dense) * p.n_tiles) * sizeof(int32_t));
 }
 
-size_t w4_stream_workspace_bytes(int64_t rows, int N, int K, int E, int epi, bool dense, int sm_count) {
+size_t w4_stream_workspace_bytes(int64_t rows, int N, int K, int E, int epi, bool dense, int sm_count,
+                                 bool zp) {
   if (rows <= 0) return 0;
   StreamPlan p = plan_stream(rows, N, K, E, epi, dense, sm_count);
-  size_t b = prep_bytes(p, rows, E, dense);
+  size_t b = prep_bytes(p, rows, E, dense, zp);
   if (p.splits > 1)
     b += counters_bytes(p, rows, E, dense) + static_cast<size_t>(p.splits) * rows * N * sizeof(float);
   return b;
 }
 
-template <int MT, int GS, bool GELU, int SCALE>
+template <int MT, int GS, bool GELU, int SCALE, bool ZP>
 static w4_status launch_one(const CUtensorMap& tmap, const CUtensorMap& smap, const w4::StreamArgs& A,
                             int sm_count, cudaStream_t stream) {
   static int attr_done[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(w4::stream_gemm_kernel<MT, GS, GELU, SCALE>,
+    if (cudaFuncSetAttribute(w4::stream_gemm_kernel<MT, GS, GELU, SCALE, ZP>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, w4::kSmemPerCta) != cudaSuccess)
       return W4_ERR_CUDA;
     attr_done[dev] = 1;
   }
-  return launch_pdl(w4::stream_gemm_kernel<MT, GS, GELU, SCALE>, dim3(sm_count), dim3(w4::kThreads),
+  return launch_pdl(w4::stream_gemm_kernel<MT, GS, GELU, SCALE, ZP>, dim3(sm_count), dim3(w4::kThreads),
                     A.L.total, stream, tmap, smap, A) == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
 template <int MT, int GS, bool GELU>
-static w4_status launch_scale(int scale_mode, const CUtensorMap& tmap, const CUtensorMap& smap,
+static w4_status launch_scale(int scale_mode, bool zp, const CUtensorMap& tmap, const CUtensorMap& smap,
                               const w4::StreamArgs& A, int sm_count, cudaStream_t stream) {
-  if (scale_mode == w4::kScaleTma) return launch_one<MT, GS, GELU, w4::kScaleTma>(tmap, smap, A, sm_count, stream);
-  if (scale_mode == w4::kScaleBlock) return launch_one<MT, GS, GELU, w4::kScaleBlock>(tmap, smap, A, sm_count, stream);
-  return launch_one<MT, GS, GELU, w4::kScaleLdg>(tmap, smap, A, sm_count, stream);
+  if (zp) return launch_one<MT, GS, GELU, w4::kScaleLdg, true>(tmap, smap, A, sm_count, stream);
+  if (scale_mode == w4::kScaleTma) return launch_one<MT, GS, GELU, w4::kScaleTma, false>(tmap, smap, A, sm_count, stream);
+  if (scale_mode == w4::kScaleBlock) return launch_one<MT, GS, GELU, w4::kScaleBlock, false>(tmap, smap, A, sm_count, stream);
+  return launch_one<MT, GS, GELU, w4::kScaleLdg, false>(tmap, smap, A, sm_count, stream);
 }
 
 template <int MT, int GS>
-static cudaError_t launch_prep(dim3 grid, size_t smem, cudaStream_t stream, const uint16_t* a,
+static cudaError_t launch_prep(bool zp, dim3 grid, size_t smem, cudaStream_t stream, const uint16_t* a,
                                const int32_t* a_row_of_pair, int kd, int64_t a_rows, int64_t rows, int K,
                                const int32_t* offsets, int E, uint8_t* xw, int n_stages, int64_t n_blocks,
                                int32_t* counters, int n_counters, int32_t* dev_status) {
-  return launch_pdl(w4::stream_prep_kernel<MT, GS>, grid, dim3(256), smem, stream, a, a_row_of_pair, kd, a_rows,
-                    rows, K, offsets, E, xw, n_stages, n_blocks, counters, n_counters, dev_status);
+  if (zp)
+    return launch_pdl(w4::stream_prep_kernel<MT, GS, true>, grid, dim3(256), smem, stream, a, a_row_of_pair, kd,
+                      a_rows, rows, K, offsets, E, xw, n_stages, n_blocks, counters, n_counters, dev_status);
+  return launch_pdl(w4::stream_prep_kernel<MT, GS, false>, grid, dim3(256), smem, stream, a, a_row_of_pair, kd,
+                    a_rows, rows, K, offsets, E, xw, n_stages, n_blocks, counters, n_counters, dev_status);
 }
 
 w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int k_div,
                                 const uint32_t* codes, const uint16_t* scales,
                                 const int32_t* offsets, int E, int64_t rows, int N, int K, int epi,
                                 uint16_t* out, void* ws, size_t ws_bytes, int32_t* dev_status,
-                                cudaStream_t stream, int sm_count, uint64_t wait_ns, int stall_after) {
+                                cudaStream_t stream, int sm_count, uint64_t wait_ns, int stall_after,
+                                const uint8_t* zeros, int group) {
   const bool dense = (offsets == nullptr);
+  const bool zp = zeros != nullptr;
+  int gshift = 0;
+  while ((32 << gshift) < group) ++gshift;
+  if ((32 << gshift) != group || K % group) return W4_ERR_INVALID_ARG;   // (callers check first)
   StreamPlan p = plan_stream(rows, N, K, E, epi, dense, sm_count);
   w4::StreamArgs A{};
   A.scales = scales; A.offsets = offsets;
   A.E = E; A.N = N; A.K = K; A.kg = K / 32; A.rows = rows; A.epi = epi; A.out = out;
+  A.zeros = zeros; A.gshift = gshift; A.kgs = K / group;
   A.splits = p.splits; A.stages_per_split = p.stages_per_split; A.n_tiles = p.n_tiles;
   A.n_stages = p.n_stages;
   A.dev_status = dev_status;
@@ -1113,7 +1178,9 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
   // direct loads.
   const bool s16 = (reinterpret_cast<uintptr_t>(scales) & 15) == 0;
   int scale_mode;
-  if (A.kg % 8 == 0 && s16) {
+  if (zp || group != 32) {
+    scale_mode = w4::kScaleLdg;            // variants: scales (and zero-points) by direct loads
+  } else if (A.kg % 8 == 0 && s16) {
     scale_mode = w4::kScaleTma;
   } else if (A.kg % 2 == 0 && A.kg <= w4::kBlockMaxKg && N % 8 == 0 && s16 &&
              (epi == W4_EPI_GELU_GATE ? (N / 2) % w4::kHalf == 0 : N % w4::kBN == 0)) {
@@ -1122,15 +1189,15 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
   } else {
     scale_mode = w4::kScaleLdg;
   }
-  A.L = make_layout(p.MT, p.GS, scale_mode, A.kg, E, p.splits > 1);
+  A.L = make_layout(p.MT, p.GS, scale_mode, A.kg, E, p.splits > 1, zp);
   if (A.L.stages < 2) return W4_ERR_UNSUPPORTED;
   if (rows == 0) return W4_OK;
-  const size_t need = w4_stream_workspace_bytes(rows, N, K, E, epi, dense, sm_count);
+  const size_t need = w4_stream_workspace_bytes(rows, N, K, E, epi, dense, sm_count, zp);
   if (ws == nullptr || ws_bytes < need) return W4_ERR_WORKSPACE;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   A.xw = wsb;
   if (p.splits > 1) {
-    uint8_t* cbase = wsb + prep_bytes(p, rows, E, dense);
+    uint8_t* cbase = wsb + prep_bytes(p, rows, E, dense, zp);
     const size_t cb = counters_bytes(p, rows, E, dense);
     A.counters = reinterpret_cast<int32_t*>(cbase);
     A.partial = reinterpret_cast<float*>(cbase + cb);
@@ -1147,9 +1214,9 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
     const int64_t nb = block_capacity(rows, p.MT, E, dense);
     const int32_t* offs = dense ? nullptr : offsets;
     const cudaError_t e = p.MT == 8
-        ? launch_prep<8, 16>(dim3(grid), psmem, stream, a, a_row_of_pair, kd, a_rows, rows, K, offs, E, wsb,
+        ? launch_prep<8, 16>(zp, dim3(grid), psmem, stream, a, a_row_of_pair, kd, a_rows, rows, K, offs, E, wsb,
                              p.n_stages, nb, A.counters, n_counters, dev_status)
-        : launch_prep<16, 8>(dim3(grid), psmem, stream, a, a_row_of_pair, kd, a_rows, rows, K, offs, E, wsb,
+        : launch_prep<16, 8>(zp, dim3(grid), psmem, stream, a, a_row_of_pair, kd, a_rows, rows, K, offs, E, wsb,
                              p.n_stages, nb, A.counters, n_counters, dev_status);
     if (e != cudaSuccess) return W4_ERR_CUDA;
   }
@@ -1161,8 +1228,8 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
     return W4_ERR_CUDA;
   const bool gelu = A.epi == W4_EPI_GELU_GATE;
   if (p.MT == 8)
-    return gelu ? launch_scale<8, 16, true>(scale_mode, tmap, smap, A, sm_count, stream)
-                : launch_scale<8, 16, false>(scale_mode, tmap, smap, A, sm_count, stream);
-  return gelu ? launch_scale<16, 8, true>(scale_mode, tmap, smap, A, sm_count, stream)
-              : launch_scale<16, 8, false>(scale_mode, tmap, smap, A, sm_count, stream);
+    return gelu ? launch_scale<8, 16, true>(scale_mode, zp, tmap, smap, A, sm_count, stream)
+                : launch_scale<8, 16, false>(scale_mode, zp, tmap, smap, A, sm_count, stream);
+  return gelu ? launch_scale<16, 8, true>(scale_mode, zp, tmap, smap, A, sm_count, stream)
+              : launch_scale<16, 8, false>(scale_mode, zp, tmap, smap, A, sm_count, stream);
 }
