@@ -258,7 +258,12 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
   int* offs = table + (A.E + 1);
   int* blk = offs + (A.E + 1);
 
-  pdl_wait();
+  // This kernel's only direct predecessor is its preparation pass, which lets it launch only
+  // once everything before the pass (the routing among it) has completed.  So the routing and
+  // the weights may be read at once: the producers issue the first lap's weight loads right away
+  // and wait for the preparation pass only before its activation copies (below), so the weight
+  // stream starts while the pass still runs.  No other thread touches memory the pass writes
+  // before it has consumed a stage that its producer issued after waiting.
 
   // unit table: table[e] = first unit of expert e, table[E] = total; offsets copied to offs[];
   // blk[e] = first token block of expert e.  Offsets that are not non-decreasing from 0 to rows
@@ -342,6 +347,23 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       return true;
     };
     auto advance = [&]() { ++issued; if (++slot == S) { slot = 0; if (!first_lap) phase ^= 1u; first_lap = false; } };
+    // the activation copies of the first lap, deferred until the preparation pass writing them
+    // has completed
+    struct Deferred { uint8_t* dst; const uint8_t* src; uint32_t bytes; uint64_t* bar; };
+    Deferred def[2 * kMaxStages];
+    int ndef = 0;
+    bool waited = false;
+    auto act_copy = [&](uint8_t* dst, const uint8_t* src, uint32_t bytes, uint64_t* bar) {
+      if (waited) bulk_g2s(dst, src, bytes, bar);
+      else def[ndef++] = Deferred{dst, src, bytes, bar};
+    };
+    auto flush = [&]() {
+      if (waited) return;
+      pdl_wait();
+      waited = true;
+      for (int i = 0; i < ndef; ++i) bulk_g2s(def[i].dst, def[i].src, def[i].bytes, def[i].bar);
+      ndef = 0;
+    };
     if (A.pf_all) {
       // weights that fit in L2 several times over: ask for all of this pipeline's code and scale
       // tiles now, so DRAM streams them at full rate while the ring fills from L2
@@ -379,6 +401,7 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       // a full block is one copy; a short block copies its rows and then the quads/multipliers
       const uint32_t xbytes = U.mt == MT ? kRec : U.mt * kXP + (kRec - kQOff);
       for (int j = U.j0; j < U.j1; ++j) {
+        if (!first_lap) flush();                // (before the first wait that can run out)
         if (!claim()) return;
         uint8_t* sl = smem + slot * L.slot_bytes;
         const int g = j * GS;
@@ -413,15 +436,16 @@ stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
         }
         const uint8_t* rec = rec0 + static_cast<int64_t>(j) * kRec;
         if (U.mt == MT) {
-          bulk_g2s(sl + kActOff, rec, kRec, &full[slot]);
+          act_copy(sl + kActOff, rec, kRec, &full[slot]);
         } else {
-          bulk_g2s(sl + kActOff, rec, U.mt * kXP, &full[slot]);
-          bulk_g2s(sl + kActOff + kQOff, rec + kQOff, kRec - kQOff, &full[slot]);
+          act_copy(sl + kActOff, rec, U.mt * kXP, &full[slot]);
+          act_copy(sl + kActOff + kQOff, rec + kQOff, kRec - kQOff, &full[slot]);
         }
         advance();
       }
     }
     // end of work: a descriptor with the done flag, completed by a plain arrive
+    flush();
     if (!claim()) return;
     StageDesc dsc{};
     dsc.bits = kDescDone << 10;
@@ -839,8 +863,10 @@ stream_prep_kernel(const uint16_t* __restrict__ a, const int32_t* __restrict__ a
   const int64_t wpb = blockDim.x >> 5;
   const int nv = K >> 3;                          // 8-element chunks in the row
   const int nblk = n_stages * kBPS;               // 256-k blocks written (zeros past K)
-  pdl_trigger();
+  // The GEMM after this pass may launch only once the kernels before the pass have completed
+  // (it reads the routing and starts its weight stream before waiting for this pass).
   pdl_wait();
+  pdl_trigger();
   // the GEMM's split-K arrival counters start at zero whatever the workspace held before
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_counters; i += gridDim.x * blockDim.x)
     counters[i] = 0;
