@@ -34,6 +34,8 @@ UNIT = "tokens/s"
 WORKLOADS = {
     "moe_decode": dict(T=64, zipf=None, name="moe_decode_T64_E128_top8_H2816_I704_g32"),
     "moe_prefill": dict(T=8192, zipf=1.1, name="moe_prefill_T8192_E128_top8_H2816_I704_g32_zipf1.1"),
+    # the dense decode GEMV of the sweep (a separate line for profiling; not the headline)
+    "dense_gemv": dict(T=16, zipf=None, name="dense_gemv_M16_K4096_N14336_g32"),
 }
 
 
@@ -234,12 +236,73 @@ def read_profile_traffic(name, src="stream_gemm.cu"):
         return None
 
 
+def native_gemv(args, world, rank, local):
+    """The dense GEMV (M = 16, K = 4096, N = 14336) as its own line: w4a16_linear calls replayed
+    from CUDA graphs over 8 rotating weight copies (264 MB, more than twice L2)."""
+    import torch
+
+    from w4a16_group_quantized_w4_b200 import api, synth
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    ranks_init(world, "nccl", device)
+    M, K, N, nc = WORKLOADS["dense_gemv"]["T"], 4096, 14336, 8
+    base = synth.case_dense_gemv(M, seed=args.seed + rank)
+    codes = [to_dev(base.codes, "u32", device) for _ in range(nc)]
+    scales = [to_dev(base.scales, "bf16", device) for _ in range(nc)]
+    x = to_dev(base.x, "bf16", device)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            api.w4a16_linear(x, codes[i % nc], scales[i % nc], y=y)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(nc):
+                api.w4a16_linear(x, codes[i], scales[i], y=y)
+        g.replay()
+    stream.synchronize()
+    reps = max(1, args.steps // nc)
+    ranks_barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    ms = ranks_max(e0.elapsed_time(e1), world, device)
+    calls = reps * nc
+    us = ms * 1e3 / calls
+    hbm_peak, _, _, peak_src = peaks()
+    byts = N * K // 2 + N * (K // 32) * 2 + M * K * 2 + M * N * 2
+    del g
+    ranks_finish(world)
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": "dense W4A16 GEMV rows/s", "value": round(job_throughput(M * calls, world, ms), 1),
+        "unit": "rows/s", "n_gpus": world, "steps": calls, "warmup": args.warmup, "ms_per_step": round(us / 1e3, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded: codes uniform over -8..7, scales 0.01|N(0,1)|+1e-4, x N(0,1))",
+        "config": {"workload": WORKLOADS["dense_gemv"]["name"], "M": M, "K": K, "N": N,
+                   "l2": f"no flush: {nc} weight copies (264 MB) rotate"},
+        "gpu_launches": 2 * calls,
+        "roofline": {"bound": "hbm", "achieved": round(byts / us / 1e3, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(byts / us / 1e3 / hbm_peak, 4), "traffic": None,
+                     "kernel": "stream_gemm_kernel with its preparation pass", "algorithmic_bytes_per_call": byts,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"},
+    }), flush=True)
+
+
 def native(args, world, rank, local):
     import numpy as np
     import torch
 
     from w4a16_group_quantized_w4_b200 import api, synth
 
+    if args.workload == "dense_gemv":
+        return native_gemv(args, world, rank, local)
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     ranks_init(world, "nccl", device)
@@ -663,6 +726,10 @@ def reference(args, world, rank):
     except Exception:
         threads = os.cpu_count()
     wl = WORKLOADS[args.workload]
+    if args.workload == "dense_gemv":
+        print(json.dumps({"impl": "reference", "unavailable": "the reference arm times the MoE workloads only"}),
+              flush=True)
+        return
     case = synth.moe_case(wl["T"], 128, 8, 2816, 704, seed=args.seed, zipf_s=wl["zipf"])
     budget_s = 150.0
 
