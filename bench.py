@@ -210,10 +210,17 @@ def gmm_bytes(counts, T, k, H, I):
     return gu, dn, hit
 
 
+# the sources a kernel is compiled from (the kernel's file, the headers holding its device code)
+KERNEL_SOURCES = {
+    "stream_gemm.cu": ["stream_gemm.cu", "stream_gemm.cuh", "common.cuh"],
+    "fused.cu": ["fused.cu", "stream_gemm.cuh", "route.cuh", "common.cuh"],
+}
+
+
 def kernel_source_hash(src="stream_gemm.cu"):
     h = hashlib.sha256()
-    p = os.path.join(ROOT, "w4a16_group_quantized_w4_b200", "csrc", src)
-    h.update(open(p, "rb").read())
+    for f in KERNEL_SOURCES.get(src, [src]):
+        h.update(open(os.path.join(ROOT, "w4a16_group_quantized_w4_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -645,8 +652,57 @@ def run_secondary(args, device, stream):
                                             "frac_bf16_peak": round(flops / ms / 1e9 / tc_peak, 3)}
         del lay
         torch.cuda.empty_cache()
+    out.update(run_fused(device, stream))
     out.update(run_stack(device, stream, L=args.stack_layers))
     return out
+
+
+def run_fused(device, stream):
+    """The single-launch fused layer (moe_w4a16_layer) against the four-call path on the decode
+    configuration at 1, 8 and 64 tokens: graph-replayed steps alternating two weight copies (856
+    MB, beyond L2), the same y bit for bit."""
+    import numpy as np
+    import torch
+
+    from w4a16_group_quantized_w4_b200 import api, synth
+    E, k, H, I = 128, 8, 2816, 704
+    case = synth.moe_case(64, E, k, H, I, seed=7)
+    W = [(to_dev(case.gu_codes, "u32", device), to_dev(case.gu_scales, "bf16", device),
+          to_dev(case.dn_codes, "u32", device), to_dev(case.dn_scales, "bf16", device)) for _ in range(2)]
+    xs, ls = to_dev(case.x, "bf16", device), to_dev(case.logits, "f32", device)
+    res = {}
+    for T in (1, 8, 64):
+        x, lg = xs[:T].contiguous(), ls[:T].contiguous()
+        row = {}
+        ys = {}
+        for name, fused in (("four_call", False), ("fused", True)):
+            lays = [api.MoELayer(*W[c], T, k, fused=fused) for c in range(2)]
+            with torch.cuda.stream(stream):
+                for i in range(3):
+                    lays[i % 2](x, lg)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for i in range(10):
+                        lays[i % 2](x, lg)
+                g.replay()
+            stream.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(30):
+                    g.replay()
+                e1.record(stream)
+            stream.synchronize()
+            row[f"{name}_us"] = round(e0.elapsed_time(e1) * 1e3 / 300, 2)
+            with torch.cuda.stream(stream):
+                ys[name] = lays[1](x, lg).clone()
+            stream.synchronize()
+            del g, lays
+        row["bit_identical"] = bool(torch.equal(ys["fused"].view(torch.int16), ys["four_call"].view(torch.int16)))
+        res[f"moe_layer_fused_vs_four_call_T{T}"] = row
+    del W
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_stack(device, stream, L=30, reps=3):
@@ -681,29 +737,32 @@ def run_stack(device, stream, L=30, reps=3):
     for T in (1, 32, 256):
         x0 = to_dev(synth.bf16_normal((T, H), 0, 600), "bf16", device)
         lgs = [to_dev(synth.router_logits(T, E, 0, 700 + l), "f32", device) for l in range(L)]
-        with torch.cuda.stream(stream):
-            for _ in range(2):
-                st.chained_step(x0, lgs, stream=stream)
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                st.chained_step(x0, lgs, stream=stream)
-            g.replay()
-        stream.synchronize()
-        hit = sum(int((torch.diff(st.layer(l, T).rt.expert_offsets) > 0).sum()) for l in range(L))
-        n = 20
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(n):
+        for fused in (False, True):
+            if fused and not st.fusable(T):
+                continue
+            with torch.cuda.stream(stream):
+                for _ in range(2):
+                    st.chained_step(x0, lgs, stream=stream, fused=fused)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    st.chained_step(x0, lgs, stream=stream, fused=fused)
                 g.replay()
-            e1.record(stream)
-        stream.synchronize()
-        ms = e0.elapsed_time(e1) / n
-        byts = hit * st.expert_bytes() + L * T * H * 2 * 2 + (L - 1) * T * H * 2 * 2   # + the chaining
-        res[f"stack_decode_{L}_layers_T{T}"] = {"ms_per_step": round(ms, 3), "tokens/s": round(T / ms * 1e3, 1),
-                                               "experts_hit": hit, "GB/s": round(byts / ms / 1e6, 1),
-                                               "frac_hbm": round(byts / ms / 1e6 / hbm_peak, 3)}
-        del g
+            stream.synchronize()
+            hit = sum(int((torch.diff(st.layer(l, T).rt.expert_offsets) > 0).sum()) for l in range(L))
+            n = 20
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(n):
+                    g.replay()
+                e1.record(stream)
+            stream.synchronize()
+            ms = e0.elapsed_time(e1) / n
+            byts = hit * st.expert_bytes() + L * T * H * 2 * 2 + (L - 1) * T * H * 2 * 2   # + the chaining
+            res[f"stack_decode_{L}_layers_T{T}" + ("_fused" if fused else "")] = {
+                "ms_per_step": round(ms, 3), "tokens/s": round(T / ms * 1e3, 1), "experts_hit": hit,
+                "GB/s": round(byts / ms / 1e6, 1), "frac_hbm": round(byts / ms / 1e6 / hbm_peak, 3)}
+            del g
     del st
     torch.cuda.empty_cache()
     return res

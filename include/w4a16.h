@@ -61,7 +61,9 @@ typedef enum {
   W4_OP_ROUTE = 2,
   W4_OP_GMM = 3,
   W4_OP_LINEAR_G = 4,       /* w4a16_linear_g (zero-points assumed present: an upper bound) */
-  W4_OP_GMM_G = 5           /* moe_w4a16_gmm_g (likewise) */
+  W4_OP_GMM_G = 5,          /* moe_w4a16_gmm_g (likewise) */
+  W4_OP_LAYER = 6,          /* moe_w4a16_layer: M_or_T = T, N = H, K = I, E, k */
+  W4_OP_LAYER_CTL = 7       /* its control area at the front of that workspace (T ignored) */
 } w4_op;
 
 /*
@@ -185,6 +187,38 @@ w4_status moe_w4a16_gmm(const uint16_t* a, const int32_t* a_row_of_pair, int32_t
  */
 w4_status moe_combine(const uint16_t* o, const float* topk_w, const int32_t* pair_pos,
                       int32_t T, int32_t k, int32_t H, uint16_t* y, void* stream);
+
+/*
+ * moe_w4a16_layer -- one MoE decode layer in ONE kernel launch:
+ *   y = moe_combine(down(gelu_gate(gate_up(x routed by logits)))),
+ * i.e. moe_route_permute, moe_w4a16_gmm (gate/up, W4_EPI_GELU_GATE), moe_w4a16_gmm (down) and
+ * moe_combine fused into a persistent kernel whose phases hand over through counters in the
+ * workspace.  ("What changed in vLLM's TPU backend": the fused-MoE layer over the experts' packed
+ * int4 weights; "The gap at 26B": 128 experts, 8 active.)  For the sizes it accepts it computes
+ * exactly what those four calls compute on the weight-streaming kernel, in the same order, so y is
+ * bit-identical to theirs.
+ *
+ *   x          [T, H] bf16, 16-byte aligned.       logits  [T, E] float32.
+ *   gu_codes   [E, 2I, H/8] uint32 (layout L1), gu_scales [E, 2I, H/32] bf16: gate rows 0..I-1
+ *              and up rows I..2I-1 of each expert.   dn_codes [E, H, I/8], dn_scales [E, H, I/32].
+ *   y          [T, H] bf16 (output, 16-byte aligned).
+ *   workspace  at least w4_workspace_bytes(W4_OP_LAYER, T, H, I, E, k) bytes, 256-byte aligned.
+ *              Its first w4_workspace_bytes(W4_OP_LAYER_CTL, 0, H, I, E, k) bytes are the
+ *              kernel's counters: zero them once before the first call (every call leaves them
+ *              zero, whatever T).  The rest holds the routing, h and the expert outputs.  Calls
+ *              sharing a workspace must not overlap on the GPU.
+ *   dev_status one int32 device word or NULL: W4_ERR_TIMEOUT if a phase's wait for another ran
+ *              out (the kernel then still ends; y is not valid), W4_ERR_INVALID_ARG as for
+ *              moe_w4a16_gmm.
+ * Accepts 1 <= T <= 128 with T * k <= 6 E (decode: the routed rows form blocks of 8 per expert),
+ * E <= 576, 1 <= k <= min(32, E), H and I multiples of 32 (T = 0: nothing to do);
+ * W4_ERR_UNSUPPORTED otherwise, W4_ERR_INVALID_ARG for malformed arguments.  The launch is
+ * cooperative (one CTA per SM, all resident); it may be captured in a CUDA graph.
+ */
+w4_status moe_w4a16_layer(const uint16_t* x, const float* logits, int32_t T, int32_t E, int32_t k,
+                          const uint32_t* gu_codes, const uint16_t* gu_scales, const uint32_t* dn_codes,
+                          const uint16_t* dn_scales, int32_t H, int32_t I, uint16_t* y, void* workspace,
+                          size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
  * w4a16_linear_g, moe_w4a16_gmm_g -- the same linear and grouped GEMM on the weight-format

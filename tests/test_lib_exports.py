@@ -52,6 +52,32 @@ def test_host_validation_rejects_bad_arguments():
     assert lib.w4_workspace_bytes(99, 1, 1, 32, 1, 1) == 0
 
 
+def test_fused_layer_sizes_and_range():
+    """moe_w4a16_layer's workspace sizing and its range checks (both before any CUDA call)."""
+    lib = _lib.load()
+    nul = C.c_void_p(None)
+    bogus = C.c_void_p(256)
+    ws = lib.w4_workspace_bytes(_lib.W4_OP_LAYER, 64, 2816, 704, 128, 8)
+    ctl = lib.w4_workspace_bytes(_lib.W4_OP_LAYER_CTL, 0, 2816, 704, 128, 8)
+    # the control area does not depend on T, and sits inside every T's workspace
+    assert ctl == lib.w4_workspace_bytes(_lib.W4_OP_LAYER_CTL, 64, 2816, 704, 128, 8)
+    assert 0 < ctl < lib.w4_workspace_bytes(_lib.W4_OP_LAYER, 1, 2816, 704, 128, 8) < ws
+    # h and o alone: 512 rows of 704 and 2816 bf16
+    assert ws > 512 * (704 + 2816) * 2
+    assert lib.w4_workspace_bytes(_lib.W4_OP_LAYER, 129, 2816, 704, 128, 8) == 0   # T > 128
+    assert lib.w4_workspace_bytes(_lib.W4_OP_LAYER, 97, 2816, 704, 128, 8) == 0    # T k > 6 E
+    assert lib.w4_workspace_bytes(_lib.W4_OP_LAYER, 96, 2816, 704, 128, 8) > ws
+    args = (bogus, bogus, bogus, bogus, 2816, 704, bogus, bogus, 1 << 30, nul, nul)
+    assert lib.moe_w4a16_layer(bogus, bogus, 129, 128, 8, *args) == _lib.W4_ERR_UNSUPPORTED
+    assert lib.moe_w4a16_layer(bogus, bogus, 97, 128, 8, *args) == _lib.W4_ERR_UNSUPPORTED
+    assert lib.moe_w4a16_layer(bogus, bogus, 4, 1024, 8, *args) == _lib.W4_ERR_UNSUPPORTED   # E > 576
+    assert lib.moe_w4a16_layer(bogus, bogus, 4, 128, 0, *args) == _lib.W4_ERR_INVALID_ARG
+    bad_h = (bogus, bogus, bogus, bogus, 2800, 704, bogus, bogus, 1 << 30, nul, nul)
+    assert lib.moe_w4a16_layer(bogus, bogus, 4, 128, 8, *bad_h) == _lib.W4_ERR_INVALID_ARG
+    assert lib.moe_w4a16_layer(nul, bogus, 4, 128, 8, *args) == _lib.W4_ERR_INVALID_ARG
+    assert lib.moe_w4a16_layer(nul, nul, 0, 128, 8, *args) == _lib.W4_OK      # nothing to do
+
+
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError):
         _lib.load(str(tmp_path / "nope.so"))

@@ -26,6 +26,8 @@ W4_OP_ROUTE = 2
 W4_OP_GMM = 3
 W4_OP_LINEAR_G = 4
 W4_OP_GMM_G = 5
+W4_OP_LAYER = 6
+W4_OP_LAYER_CTL = 7
 
 # name -> (restype, argtypes), mirroring include/w4a16.h
 _P = C.c_void_p
@@ -44,6 +46,7 @@ SIGNATURES = {
     "w4a16_linear_g": (_I32, [_P, _P, _P, _P, _I32, _P, _I64, _I64, _I64, _P, _SZ, _P]),
     "moe_w4a16_gmm_g": (_I32, [_P, _P, _I32, _P, _P, _P, _I32, _P, _I32, _I64, _I32, _I32, _I32, _P,
                                _P, _SZ, _P, _P]),
+    "moe_w4a16_layer": (_I32, [_P, _P, _I32, _I32, _I32, _P, _P, _P, _P, _I32, _I32, _P, _P, _SZ, _P, _P]),
     "w4_workspace_bytes": (_SZ, [_I32, _I64, _I64, _I64, _I32, _I32]),
     "w4_status_str": (C.c_char_p, [_I32]),
     "w4_last_cuda_error": (_I32, []),

@@ -277,18 +277,68 @@ def moe_w4a16_gmm_g(a, a_row_of_pair, k: int, codes, scales, expert_offsets, row
     return out
 
 
+def moe_layer_fusable(T: int, E: int, k: int, H: int, I: int) -> bool:
+    """Whether moe_w4a16_layer accepts these sizes (1 <= T <= 128, T k <= 6 E, E <= 576)."""
+    return T >= 1 and w4_workspace_bytes(_lib.W4_OP_LAYER, T, H, I, E, k) > 0
+
+
+def layer_workspace(T: int, E: int, k: int, H: int, I: int, device) -> torch.Tensor:
+    """A private workspace for moe_w4a16_layer, zero-filled (its control area must start at
+    zero; every call leaves it so).  Not shared with other calls."""
+    nbytes = w4_workspace_bytes(_lib.W4_OP_LAYER, T, H, I, E, k)
+    if nbytes == 0:
+        raise _lib.W4Error("moe_w4a16_layer", _lib.W4_ERR_UNSUPPORTED)
+    return torch.zeros((nbytes + 255) // 256 * 256, dtype=torch.uint8, device=device)
+
+
+def moe_w4a16_layer(x, logits, k: int, gu_codes, gu_scales, dn_codes, dn_scales, y=None, ws=None,
+                    dev_status=None, stream=None):
+    """One MoE decode layer in one kernel launch: x bf16 [T, H], logits f32 [T, E], gate/up
+    codes [E, 2I, H/8] / scales [E, 2I, H/32], down codes [E, H, I/8] / scales [E, H, I/32]
+    -> y bf16 [T, H].  ws: a workspace from layer_workspace (allocated here when None)."""
+    lib = _lib.load()
+    T, H = x.shape
+    E, N2, _ = gu_codes.shape
+    I = N2 // 2
+    dev = x.device
+    _need("x", x, torch.bfloat16, (T, H), dev)
+    _need("logits", logits, torch.float32, (T, E), dev)
+    _need("gu_codes", gu_codes, torch.int32, (E, 2 * I, H // 8), dev)
+    _need("gu_scales", gu_scales, torch.bfloat16, (E, 2 * I, H // 32), dev)
+    _need("dn_codes", dn_codes, torch.int32, (E, H, I // 8), dev)
+    _need("dn_scales", dn_scales, torch.bfloat16, (E, H, I // 32), dev)
+    y = torch.empty((T, H), dtype=torch.bfloat16, device=dev) if y is None else y
+    _need("y", y, torch.bfloat16, (T, H), dev)
+    if ws is None:
+        ws = layer_workspace(T, E, k, H, I, dev)
+    _need("ws", ws, torch.uint8, None, dev)
+    if dev_status is not None:
+        _need("dev_status", dev_status, torch.int32, (1,), dev)
+    _lib.check("moe_w4a16_layer", lib.moe_w4a16_layer(
+        _p(x), _p(logits), T, E, k, _p(gu_codes), _p(gu_scales), _p(dn_codes), _p(dn_scales), H, I,
+        _p(y), _p(ws), ws.numel(), _p(dev_status), _s(stream)))
+    return y
+
+
 class MoELayer:
     """One mixture-of-experts layer on the device: the four entry points composed on one stream
     (route -> gate/up GEMM with the GELU gate -> down GEMM -> combine), with every buffer
-    allocated once so that a step launches kernels only."""
+    allocated once so that a step launches kernels only.  fused=True runs the same layer as one
+    moe_w4a16_layer launch (decode sizes only; its routing, h and o then stay in the layer's
+    private workspace)."""
 
-    def __init__(self, gu_codes, gu_scales, dn_codes, dn_scales, T: int, k: int):
+    def __init__(self, gu_codes, gu_scales, dn_codes, dn_scales, T: int, k: int, fused: bool = False):
         self.E, self.N2, _ = gu_codes.shape
         self.H = gu_codes.shape[2] * 8
         self.I = self.N2 // 2
         self.T, self.k = T, k
         dev = gu_codes.device
         self.w = (gu_codes, gu_scales, dn_codes, dn_scales)
+        self.fused = fused
+        if fused:
+            self.layer_ws = layer_workspace(T, self.E, k, self.H, self.I, dev)
+            self.y = torch.empty((T, self.H), dtype=torch.bfloat16, device=dev)
+            return
         self.rt = Routing(torch.empty((T, k), dtype=torch.int32, device=dev),
                           torch.empty((T, k), dtype=torch.float32, device=dev),
                           torch.empty(self.E + 1, dtype=torch.int32, device=dev),
@@ -303,6 +353,9 @@ class MoELayer:
 
     def __call__(self, x, logits, stream=None):
         gu_c, gu_s, dn_c, dn_s = self.w
+        if self.fused:
+            return moe_w4a16_layer(x, logits, self.k, gu_c, gu_s, dn_c, dn_s, y=self.y,
+                                   ws=self.layer_ws, stream=stream)
         moe_route_permute(logits, self.k, out=self.rt, ws=self.route_ws, stream=stream)
         moe_w4a16_gmm(x, self.rt.sorted_pair, self.k, gu_c, gu_s, self.rt.expert_offsets,
                       self.T * self.k, W4_EPI_GELU_GATE, out=self.h, stream=stream)

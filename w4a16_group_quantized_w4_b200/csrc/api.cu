@@ -27,6 +27,13 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
                                 cudaStream_t stream, int sm_count, uint64_t wait_ns = 0,
                                 int stall_after = -1, const uint8_t* zeros = nullptr, int group = 32);
 size_t w4_tc_workspace_bytes(int64_t rows, int K, int64_t wrows);
+size_t w4_layer_workspace_bytes(int T, int E, int k, int H, int I, int sm_count);
+size_t w4_layer_control_bytes(int E, int k, int H, int I, int sm_count);
+w4_status w4_layer_check(int T, int E, int k, int H, int I);
+w4_status w4_launch_moe_layer(const uint16_t* x, const float* logits, int T, int E, int k,
+                              const uint32_t* gu_codes, const uint16_t* gu_scales, const uint32_t* dn_codes,
+                              const uint16_t* dn_scales, int H, int I, uint16_t* y, void* ws, size_t ws_bytes,
+                              int32_t* dev_status, cudaStream_t stream, int sm_count);
 bool w4_tm_supported(int N, int K, int epi);
 w4_status w4_launch_tm_gemm(const uint16_t* a, const int32_t* a_row_of_pair, int k_div,
                             const uint32_t* codes, const uint16_t* scales, const int32_t* offsets,
@@ -132,6 +139,13 @@ size_t w4_workspace_bytes(int32_t op, int64_t M_or_T, int64_t N, int64_t K, int3
         }
         return need;
       }
+    case W4_OP_LAYER:
+    case W4_OP_LAYER_CTL:
+      if (M_or_T > (1LL << 30) || N > (1LL << 30) || K > (1LL << 30)) return 0;
+      if (op == W4_OP_LAYER)
+        return w4_layer_workspace_bytes(static_cast<int>(M_or_T), E, k, static_cast<int>(N), static_cast<int>(K),
+                                        current_sm_count());
+      return w4_layer_control_bytes(E, k, static_cast<int>(N), static_cast<int>(K), current_sm_count());
     default:
       return 0;
   }
@@ -269,6 +283,22 @@ w4_status moe_w4a16_gmm_g(const uint16_t* a, const int32_t* a_row_of_pair, int32
                                       epilogue, out, workspace, workspace_bytes, dev_status,
                                       static_cast<cudaStream_t>(stream), current_sm_count(), 0, -1, zeros,
                                       group));
+}
+
+w4_status moe_w4a16_layer(const uint16_t* x, const float* logits, int32_t T, int32_t E, int32_t k,
+                          const uint32_t* gu_codes, const uint16_t* gu_scales, const uint32_t* dn_codes,
+                          const uint16_t* dn_scales, int32_t H, int32_t I, uint16_t* y, void* workspace,
+                          size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  const w4_status chk = w4_layer_check(T, E, k, H, I);
+  if (chk != W4_OK) return chk;
+  if (T == 0) return W4_OK;
+  if (!x || !logits || !gu_codes || !gu_scales || !dn_codes || !dn_scales || !y) return W4_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(y, 16) || !aligned(gu_codes, 16) || !aligned(dn_codes, 16) ||
+      !aligned(gu_scales, 4) || !aligned(dn_scales, 4) || (workspace && !aligned(workspace, 256)))
+    return W4_ERR_INVALID_ARG;
+  return finish(w4_launch_moe_layer(x, logits, T, E, k, gu_codes, gu_scales, dn_codes, dn_scales, H, I, y,
+                                    workspace, workspace_bytes, dev_status, static_cast<cudaStream_t>(stream),
+                                    current_sm_count()));
 }
 
 w4_status moe_combine(const uint16_t* o, const float* topk_w, const int32_t* pair_pos, int32_t T,

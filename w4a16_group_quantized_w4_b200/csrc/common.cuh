@@ -47,6 +47,10 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
 }
 
+__device__ __forceinline__ void mbar_inval(uint64_t* bar) {
+  asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
@@ -255,6 +259,37 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 
 __device__ __forceinline__ void set_status(int32_t* dev_status, int32_t code) {
   if (dev_status) atomicCAS(dev_status, 0, code);
+}
+
+// ------------------------------------------------------------------------------------------
+// hand-over between CTAs of one kernel: counters in global memory
+// ------------------------------------------------------------------------------------------
+
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// orders this thread's generic-proxy global accesses with later async-proxy ones (bulk copies)
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// orders this thread's generic-proxy shared-memory accesses with later async-proxy ones
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Bounded wait until *p >= need (acquire at GPU scope); false once limit_ns have passed.
+__device__ __forceinline__ bool wait_count(const int32_t* p, int need, uint64_t limit_ns) {
+  if (ld_acquire_gpu(p) >= need) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(32);
+    if (ld_acquire_gpu(p) >= need) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
 }
 
 }  // namespace w4

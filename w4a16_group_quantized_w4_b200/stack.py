@@ -65,34 +65,40 @@ class MoEStack:
         return RepackReport(int(o[0]), int(o[1]), g_gu, g_dn)
 
     # ------------------------------------------------------------------ decode
-    def layer(self, l: int, T: int) -> api.MoELayer:
-        """The four-call MoE layer l for T tokens (buffers allocated once per (l, T))."""
-        key = (l, T)
+    def fusable(self, T: int) -> bool:
+        """Whether T tokens fit the single-launch fused layer (moe_w4a16_layer)."""
+        return api.moe_layer_fusable(T, self.E, self.k, self.H, self.I)
+
+    def layer(self, l: int, T: int, fused: bool = False) -> api.MoELayer:
+        """MoE layer l for T tokens (buffers allocated once per (l, T, fused)): the four-call
+        path, or the single-launch fused layer when fused and T fits it."""
+        fused = fused and self.fusable(T)
+        key = (l, T, fused)
         if key not in self._layers:
             self._layers[key] = api.MoELayer(self.gu_codes[l], self.gu_scales[l], self.dn_codes[l],
-                                             self.dn_scales[l], T, self.k)
+                                             self.dn_scales[l], T, self.k, fused=fused)
         return self._layers[key]
 
-    def step(self, xs, logits, stream=None):
+    def step(self, xs, logits, stream=None, fused: bool = False):
         """One decode step through every layer with independent inputs: xs[l] bf16 [T, H],
         logits[l] f32 [T, E] -> the list of layer outputs y_l bf16 [T, H] (each layer's own
         buffer)."""
         T = xs[0].shape[0]
-        return [self.layer(l, T)(xs[l], logits[l], stream=stream) for l in range(self.L)]
+        return [self.layer(l, T, fused)(xs[l], logits[l], stream=stream) for l in range(self.L)]
 
-    def chained_step(self, x0, logits, stream=None):
+    def chained_step(self, x0, logits, stream=None, fused: bool = False):
         """One decode step through the chained stack: layer 0 takes x0 bf16 [T, H]; layer l + 1
         takes moe_rms_chain(y_l).  Returns (the inputs x_l, the outputs y_l), device buffers
-        owned by the stack (overwritten by the next chained step of the same T)."""
+        owned by the stack (overwritten by the next chained step of the same T and path)."""
         T = x0.shape[0]
-        key = ("chain", T)
+        key = ("chain", T, fused)
         if key not in self._layers:
             self._layers[key] = [torch.empty((T, self.H), dtype=torch.bfloat16, device=x0.device)
                                  for _ in range(self.L - 1)]
         xb = self._layers[key]
         xs, ys = [x0], []
         for l in range(self.L):
-            y = self.layer(l, T)(xs[l], logits[l], stream=stream)
+            y = self.layer(l, T, fused)(xs[l], logits[l], stream=stream)
             ys.append(y)
             if l + 1 < self.L:
                 xs.append(api.moe_rms_chain(y, x_next=xb[l], stream=stream))
