@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--stack-layers", type=int, default=30,
                     help="layers of the secondary repack + expert-stack measurement (30: the full stack)")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--path", choices=["four_call", "fused"], default="four_call",
+                    help="decode layer as four calls (six kernels) or as the single-launch fused layer")
     return ap.parse_args()
 
 
@@ -316,11 +318,15 @@ def native(args, world, rank, local):
     wl = WORKLOADS[args.workload]
     T, E, k, H, I = wl["T"], 128, 8, 2816, 704
     case = synth.moe_case(T, E, k, H, I, seed=args.seed + rank, zipf_s=wl["zipf"])
+    fused = args.path == "fused"
+    if fused and not api.moe_layer_fusable(T, E, k, H, I):
+        raise SystemExit(f"--path fused: {wl['name']} is outside the fused layer's range")
     copies = 2
     layers = []
     for c in range(copies):
         layers.append(api.MoELayer(to_dev(case.gu_codes, "u32", device), to_dev(case.gu_scales, "bf16", device),
-                                   to_dev(case.dn_codes, "u32", device), to_dev(case.dn_scales, "bf16", device), T, k))
+                                   to_dev(case.dn_codes, "u32", device), to_dev(case.dn_scales, "bf16", device), T, k,
+                                   fused=fused))
     x = to_dev(case.x, "bf16", device)
     logits = to_dev(case.logits, "f32", device)
     stream = torch.cuda.Stream(device)
@@ -386,7 +392,9 @@ def native(args, world, rank, local):
     # graph-replayed step, without its other kernels.
     lay = layers[0]
     with torch.cuda.stream(stream):
-        api.moe_route_permute(logits, k, out=lay.rt, ws=lay.route_ws)
+        rt = api.moe_route_permute(logits, k)
+        if not fused:
+            api.moe_route_permute(logits, k, out=lay.rt, ws=lay.route_ws)
     stream.synchronize()
     n_k = 20
 
@@ -404,7 +412,7 @@ def native(args, world, rank, local):
         return g
 
     t_k = {}
-    for which in ("gu", "dn"):
+    for which in (() if fused else ("gu", "dn")):
         g = gemm_graph(which)
         with torch.cuda.stream(stream):
             g.replay()
@@ -419,15 +427,26 @@ def native(args, world, rank, local):
         stream.synchronize()
         t_k[which] = e0.elapsed_time(e1) / 1e3 / (reps * n_k)
         del g
-    t_gu, t_dn = t_k["gu"], t_k["dn"]
-    counts = np.diff(lay.rt.expert_offsets.cpu().numpy())
+    t_gu, t_dn = t_k.get("gu", 0.0), t_k.get("dn", 0.0)
+    counts = np.diff(rt.expert_offsets.cpu().numpy())
     b_gu, b_dn, hit = gmm_bytes(counts, T, k, H, I)
     hbm_peak, tc_peak, tc_sus, peak_src = peaks()
     prefill = args.workload == "moe_prefill"
     # kernels per step: decode = route, (preparation pass + GEMM) x 2, combine; prefill = two-launch
     # route, (conversion + weight-row exponents + GEMM) x 2, combine
-    kernels = 9 if prefill else 6
-    if prefill:
+    kernels = 9 if prefill else (1 if fused else 6)
+    if fused:
+        # one launch per step: the fused kernel's roofline is the step's algorithmic bytes over the
+        # step time (its routing, preparation and combine phases included)
+        t_step = ms_per_step / 1e3
+        achieved = (b_gu + b_dn) / t_step / 1e9
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                    "frac": round(achieved / hbm_peak, 4),
+                    "traffic": read_profile_traffic("fused_layer_moe_decode.md", "fused.cu"),
+                    "kernel": "moe_layer_kernel (the whole step: one cooperative launch, graph-replayed)",
+                    "algorithmic_bytes_per_step": int(b_gu + b_dn), "experts_hit": hit,
+                    "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"}
+    elif prefill:
         # many routed rows per expert: the tensor-memory kernel, a tensor-core roofline on the
         # GEMMs' algorithmic FLOPs (each launch timed alone: the burst peak)
         flops = 2.0 * T * k * (2 * I * H + H * I)
@@ -500,13 +519,16 @@ def native(args, world, rank, local):
                    "hidden": H, "intermediate": I, "group": 32, "parallelism": f"replicas{world}",
                    "l2": f"no flush: {copies} weight copies of 428 MB alternate, each step streams the "
                          f"{hit} experts hit (>126 MB L2)",
-                   "timing": f"CUDA graphs of {spg} consecutive steps (4 calls, {kernels} kernels each; weight copies "
-                             f"alternating), replayed {args.steps // spg} times; CUDA events on the launch stream"},
+                   "path": args.path,
+                   "timing": f"CUDA graphs of {spg} consecutive steps ({'1 fused call' if fused else '4 calls'}, "
+                             f"{kernels} kernel(s) each; weight copies alternating), replayed {args.steps // spg} "
+                             f"times; CUDA events on the launch stream"},
         "clocks": clocks.summary(),
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT,
                 "h2d_bytes_per_step": int(x.numel() * 2 + logits.numel() * 4),
                 "d2h_bytes_per_step": int(T * H * 2),
-                "how": f"public API (MoELayer) per step: pinned H2D of x and logits, 4 calls ({kernels} kernels), D2H of y"},
+                "how": f"public API (MoELayer) per step: pinned H2D of x and logits, "
+                       f"{'1 fused call' if fused else '4 calls'} ({kernels} kernel(s)), D2H of y"},
         "gpu_launches": kernels * args.steps,
         "step_time_distribution": step_dist,
         "roofline": roofline,

@@ -21,7 +21,7 @@
 
 namespace w4 {
 
-__global__ void __launch_bounds__(kFusedWarps * 32) route_fused_kernel(const __grid_constant__ RouteArgs A) {
+__global__ void __launch_bounds__(kFusedWarps * 32) route_fused_kernel(RouteArgs A) {
   extern __shared__ int smem[];
   route_fused_body<true>(A, smem);
 }

@@ -181,7 +181,7 @@ static __device__ void scatter_pairs(const RouteArgs& A, int64_t p0, int64_t p1,
 // FROM_IDS: the top-k is already in topk_ids / topk_w (written earlier in the same kernel by
 // route_topk_one); only the offsets and the permutation are formed here.
 template <bool PDL, bool FROM_IDS = false>
-__device__ __forceinline__ void route_fused_body(const RouteArgs& A, int* smem) {
+__device__ __forceinline__ void route_fused_body(const RouteArgs A, int* smem) {
   const int W = (A.T + 31) >> 5;                          // mask words per expert (<= 4)
   uint32_t* s_mask = reinterpret_cast<uint32_t*>(smem);   // [E][W]
   int* s_off = smem + A.E * W;                            // [E]

@@ -4,6 +4,8 @@
 
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -87,9 +89,10 @@ struct StreamArgs {
   int32_t* dev_status;
   uint64_t wait_ns;         // limit of every bounded wait
   int stall_after;          // fault injection for tests: producers stop after this many stages (< 0: never)
-  // Hand-over inside one kernel (the fused MoE decode kernel; null otherwise): the producers copy
-  // a token block's records only once act_ready[block] has reached the block's row count, and
-  // every finished (block, weight tile) adds one to tile_done[block] once its outputs are written.
+  // Hand-over inside one kernel (the fused MoE decode kernel, which instantiates the body with
+  // HO = true; unused otherwise): the producers copy a token block's records only once
+  // act_ready[block] has reached the block's row count, and every finished (block, weight tile)
+  // adds one to tile_done[block] once its outputs are written.
   const int32_t* act_ready;
   int32_t* tile_done;
 };
@@ -191,11 +194,12 @@ struct NoPreWork {
 };
 
 // The kernel's body (stream_gemm_kernel, and two phases of the fused MoE decode kernel): smem_raw
-// is the dynamic shared memory of the CTA.  pre(offs, blk, w, n) runs on the n = 16 compute warps
-// (w = 0..15) once the unit table is built and before they consume the first stage, while the
-// producers already stream weights: offs / blk are the table's per-expert row offsets and first
-// token blocks (shared memory).  It may use warp-level synchronisation only.
-template <int MT, int GS, bool GELU, int SCALE, bool ZP, typename Pre = NoPreWork>
+// is the dynamic shared memory of the CTA.  HO: the in-kernel hand-over through A.act_ready /
+// A.tile_done is compiled in.  pre(offs, blk, w, n) runs on the n = 16 compute warps (w = 0..15)
+// once the unit table is built and before they consume the first stage, while the producers
+// already stream weights: offs / blk are the table's per-expert row offsets and first token
+// blocks (shared memory).  It may use warp-level synchronisation only.
+template <int MT, int GS, bool GELU, int SCALE, bool ZP, bool HO = false, typename Pre = NoPreWork>
 __device__ __forceinline__ void stream_gemm_body(const CUtensorMap& tmap_codes, const CUtensorMap& tmap_scales,
                                                  const StreamArgs& A, uint8_t* smem_raw, const Pre& pre = Pre{}) {
   constexpr int kActOff = slot_act_off(GS);
@@ -235,25 +239,23 @@ __device__ __forceinline__ void stream_gemm_body(const CUtensorMap& tmap_codes, 
 
   // unit table: table[e] = first unit of expert e, table[E] = total; offsets copied to offs[];
   // blk[e] = first token block of expert e.  Offsets that are not non-decreasing from 0 to rows
-  // make the launch a no-op (W4_ERR_INVALID_ARG).  The offsets come into shared memory with one
-  // load per thread (a single round trip to memory); warp 0 then forms the table from there.
-  for (int e = threadIdx.x; e <= A.E; e += blockDim.x)
-    offs[e] = A.offsets ? A.offsets[e] : (e == 0 ? 0 : static_cast<int>(A.rows));
-  __syncthreads();
+  // make the launch a no-op (W4_ERR_INVALID_ARG).
   if (warp_all == 0) {
     int run = 0, brun = 0;
     bool bad = false;
-    if (A.offsets && lane == 0) bad = (offs[0] != 0) || (offs[A.E] != A.rows);
+    if (A.offsets && lane == 0) bad = (A.offsets[0] != 0) || (A.offsets[A.E] != A.rows);
     for (int base = 0; base < A.E; base += 32) {
       const int e = base + lane;
       int cnt = 0, nb = 0;
       if (e < A.E) {
-        const int64_t o0 = A.offsets ? offs[e] : 0;
-        const int64_t o1 = A.offsets ? offs[e + 1] : A.rows;
+        const int64_t o0 = A.offsets ? A.offsets[e] : 0;
+        const int64_t o1 = A.offsets ? A.offsets[e + 1] : A.rows;
         if (o1 < o0 || o0 < 0 || o1 > A.rows) bad = true;
         const int64_t ntb = o1 > o0 ? (o1 - o0 + MT - 1) / MT : 0;
         nb = static_cast<int>(ntb);
         cnt = static_cast<int>(ntb * A.n_tiles * A.splits);
+        offs[e] = static_cast<int>(o0);
+        if (e == A.E - 1) offs[A.E] = static_cast<int>(o1);
       }
       int incl = cnt, bincl = nb;
 #pragma unroll
@@ -319,7 +321,9 @@ __device__ __forceinline__ void stream_gemm_body(const CUtensorMap& tmap_codes, 
     auto advance = [&]() { ++issued; if (++slot == S) { slot = 0; if (!first_lap) phase ^= 1u; first_lap = false; } };
     // the activation copies of the first lap, deferred until the preparation pass writing them
     // has completed
-    struct Deferred { uint8_t* dst; const uint8_t* src; uint32_t bytes; uint64_t* bar; int blk, need; };
+    struct DeferredPlain { uint8_t* dst; const uint8_t* src; uint32_t bytes; uint64_t* bar; };
+    struct DeferredHO { uint8_t* dst; const uint8_t* src; uint32_t bytes; uint64_t* bar; int blk, need; };
+    using Deferred = typename std::conditional<HO, DeferredHO, DeferredPlain>::type;
     Deferred def[2 * kMaxStages];
     int ndef = 0;
     bool waited = false;
@@ -329,7 +333,7 @@ __device__ __forceinline__ void stream_gemm_body(const CUtensorMap& tmap_codes, 
     int ready_blk = -1;
     bool ready_gave_up = false;
     auto ready_wait = [&](int b, int need) {
-      if (!A.act_ready || b == ready_blk || ready_gave_up) return;
+      if (!HO || !A.act_ready || b == ready_blk || ready_gave_up) return;
       if (!wait_count(A.act_ready + b, need, A.wait_ns)) {
         set_status(A.dev_status, W4_ERR_TIMEOUT);
         ready_gave_up = true;
@@ -342,7 +346,8 @@ __device__ __forceinline__ void stream_gemm_body(const CUtensorMap& tmap_codes, 
         ready_wait(b, need);
         bulk_g2s(dst, src, bytes, bar);
       } else {
-        def[ndef++] = Deferred{dst, src, bytes, bar, b, need};
+        if constexpr (HO) def[ndef++] = Deferred{dst, src, bytes, bar, b, need};
+        else def[ndef++] = Deferred{dst, src, bytes, bar};
       }
     };
     auto flush = [&]() {
@@ -350,7 +355,7 @@ __device__ __forceinline__ void stream_gemm_body(const CUtensorMap& tmap_codes, 
       pdl_wait();
       waited = true;
       for (int i = 0; i < ndef; ++i) {
-        ready_wait(def[i].blk, def[i].need);
+        if constexpr (HO) ready_wait(def[i].blk, def[i].need);
         bulk_g2s(def[i].dst, def[i].src, def[i].bytes, def[i].bar);
       }
       ndef = 0;
@@ -407,7 +412,7 @@ __device__ __forceinline__ void stream_gemm_body(const CUtensorMap& tmap_codes, 
         dsc.e = U.e;
         dsc.sp = U.sp;
         dsc.tile = U.tile;
-        dsc.blk = U.blk;
+        dsc.blk = HO ? U.blk : 0;
         *reinterpret_cast<StageDesc*>(sl + kDescOff) = dsc;
         // the arrive releases the descriptor written above
         mbar_arrive_expect_tx(&full[slot], nbox * 2 * kBoxBytes + sbytes + xbytes);
@@ -650,7 +655,7 @@ __device__ __forceinline__ void stream_gemm_body(const CUtensorMap& tmap_codes, 
     const bool last = dflags & kDescLast;
     int sp_last = 0, tile_last = 0, blk_last = 0;   // the unit's K split, tile id, token block
     if (last) {
-      if (A.splits > 1 || A.tile_done) {
+      if (A.splits > 1 || HO) {
         const int4 d1 = *reinterpret_cast<const int4*>(sp8 + kDescOff + 16);   // before the slot is freed
         sp_last = d1.y;
         tile_last = d1.z;
@@ -731,7 +736,7 @@ __device__ __forceinline__ void stream_gemm_body(const CUtensorMap& tmap_codes, 
           }
         }
       }
-      if (A.tile_done) {
+      if (HO && A.tile_done) {
         // hand-over: once the warps have met, one thread makes their outputs visible GPU-wide
         // (a fence after the meeting covers every write ordered before it) and moves the count
         if (!epi_sync()) return;
@@ -824,7 +829,7 @@ __device__ __forceinline__ void stream_gemm_body(const CUtensorMap& tmap_codes, 
         }
       }
       if (!epi_sync()) return;
-      if (A.tile_done && flags[1] && ctid == 0) {
+      if (HO && A.tile_done && flags[1] && ctid == 0) {
         __threadfence();
         atomicAdd(A.tile_done + blk_last, 1);
       }
