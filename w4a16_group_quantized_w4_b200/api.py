@@ -46,17 +46,25 @@ def _need(name, t, dtype, shape=None, dev=None):
 _WS: dict = {}
 
 
-def workspace(nbytes: int, device) -> torch.Tensor | None:
-    """A scratch buffer of at least nbytes, cached per device and shared by calls on it (the
-    library clears what it relies on, so contents left by earlier calls do not matter)."""
+def workspace(nbytes: int, device, stream=None) -> torch.Tensor | None:
+    """A scratch buffer of at least nbytes for calls on (device, stream).
+
+    One buffer per stream: calls on one stream run in order, so they may share it (the library
+    clears what it relies on, so contents left by earlier calls do not matter), while calls on
+    different streams never do.  A buffer that is outgrown is kept alive, not freed, so a CUDA
+    graph captured with it stays valid; a capture on its own stream gets its own buffer.
+    """
     if nbytes == 0:
         return None
-    key = torch.device(device)
-    buf = _WS.get(key)
-    if buf is None or buf.numel() < nbytes:
-        buf = torch.zeros((nbytes + 255) // 256 * 256, dtype=torch.uint8, device=key)
-        _WS[key] = buf
-    return buf
+    dev = torch.device(device)
+    if dev.index is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    key = (dev, s.cuda_stream)
+    bufs = _WS.setdefault(key, [])
+    if not bufs or bufs[-1].numel() < nbytes:
+        bufs.append(torch.zeros((nbytes + 255) // 256 * 256, dtype=torch.uint8, device=dev))
+    return bufs[-1]
 
 
 def w4_workspace_bytes(op: int, m_or_t: int, n: int, k_dim: int, e: int, k: int) -> int:
@@ -97,7 +105,7 @@ def w4a16_linear(x, codes, scales, y=None, ws=None, stream=None):
     _need("y", y, torch.bfloat16, (M, N), dev)
     nbytes = w4_workspace_bytes(_lib.W4_OP_LINEAR, M, N, K, 1, 1)
     if ws is None:
-        ws = workspace(nbytes, dev)
+        ws = workspace(nbytes, dev, stream)
     _lib.check("w4a16_linear", lib.w4a16_linear(_p(x), _p(codes), _p(scales), _p(y), M, N, K,
                                                 _p(ws), 0 if ws is None else ws.numel(), _s(stream)))
     return y
@@ -118,7 +126,7 @@ def w4a16_linear_g(x, codes, scales, group: int, zeros=None, y=None, ws=None, st
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev) if y is None else y
     _need("y", y, torch.bfloat16, (M, N), dev)
     if ws is None:
-        ws = workspace(w4_workspace_bytes(_lib.W4_OP_LINEAR_G, M, N, K, 1, 1), dev)
+        ws = workspace(w4_workspace_bytes(_lib.W4_OP_LINEAR_G, M, N, K, 1, 1), dev, stream)
     _lib.check("w4a16_linear_g", lib.w4a16_linear_g(_p(x), _p(codes), _p(scales), _p(zeros), group, _p(y),
                                                     M, N, K, _p(ws), 0 if ws is None else ws.numel(),
                                                     _s(stream)))
@@ -176,7 +184,7 @@ def moe_route_permute(logits, k: int, out: Routing | None = None, ws=None, strea
     _need("pair_pos", out.pair_pos, torch.int32, (T * k,), dev)
     nbytes = w4_workspace_bytes(_lib.W4_OP_ROUTE, T, 0, 0, E, k)
     if ws is None:
-        ws = workspace(nbytes, dev)
+        ws = workspace(nbytes, dev, stream)
     _lib.check("moe_route_permute", lib.moe_route_permute(
         _p(logits), T, E, k, _p(out.topk_ids), _p(out.topk_w), _p(out.expert_offsets),
         _p(out.sorted_pair), _p(out.pair_pos), _p(ws), 0 if ws is None else ws.numel(), _s(stream)))
@@ -203,7 +211,7 @@ def moe_w4a16_gmm(a, a_row_of_pair, k: int, codes, scales, expert_offsets, rows:
     _need("out", out, torch.bfloat16, (rows, n_out), dev)
     nbytes = w4_workspace_bytes(_lib.W4_OP_GMM, rows, N, K, E, k)
     if ws is None:
-        ws = workspace(nbytes, dev)
+        ws = workspace(nbytes, dev, stream)
     if dev_status is not None:
         _need("dev_status", dev_status, torch.int32, (1,), dev)
     _lib.check("moe_w4a16_gmm", lib.moe_w4a16_gmm(
@@ -267,7 +275,7 @@ def moe_w4a16_gmm_g(a, a_row_of_pair, k: int, codes, scales, expert_offsets, row
     out = torch.empty((rows, n_out), dtype=torch.bfloat16, device=dev) if out is None else out
     _need("out", out, torch.bfloat16, (rows, n_out), dev)
     if ws is None:
-        ws = workspace(w4_workspace_bytes(_lib.W4_OP_GMM_G, rows, N, K, E, k), dev)
+        ws = workspace(w4_workspace_bytes(_lib.W4_OP_GMM_G, rows, N, K, E, k), dev, stream)
     if dev_status is not None:
         _need("dev_status", dev_status, torch.int32, (1,), dev)
     _lib.check("moe_w4a16_gmm_g", lib.moe_w4a16_gmm_g(
@@ -347,9 +355,9 @@ class MoELayer:
         self.h = torch.empty((T * k, self.I), dtype=torch.bfloat16, device=dev)
         self.o = torch.empty((T * k, self.H), dtype=torch.bfloat16, device=dev)
         self.y = torch.empty((T, self.H), dtype=torch.bfloat16, device=dev)
-        self.route_ws = workspace(w4_workspace_bytes(_lib.W4_OP_ROUTE, T, 0, 0, self.E, k), dev)
-        if self.route_ws is not None:
-            self.route_ws = self.route_ws.clone()   # private: layers may run back to back
+        nr = w4_workspace_bytes(_lib.W4_OP_ROUTE, T, 0, 0, self.E, k)
+        # private: the routing outputs of layers that run back to back must not share scratch
+        self.route_ws = torch.zeros(nr, dtype=torch.uint8, device=dev) if nr else None
 
     def __call__(self, x, logits, stream=None):
         gu_c, gu_s, dn_c, dn_s = self.w

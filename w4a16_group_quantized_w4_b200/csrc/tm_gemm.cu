@@ -310,6 +310,7 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
     int slot = 0;
     uint32_t ph = 0;
     bool lap0 = true, ok = true;
+    int64_t issued = 0;                        // code stages issued (lane 0)
     for (int t = blockIdx.x; t < total && ok && !*abort_flag; t += gridDim.x) {
       if (lane == 0) {
         if (t == static_cast<int>(blockIdx.x)) prefetch_tmap(&tmap_codes);
@@ -323,12 +324,19 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
           mbar_arrive_expect_tx(&cfull[slot], C::kCodeStage);
           tma_load_2d(cdst, &tmap_codes, st * (KSK / 8), row_a, &cfull[slot]);
           tma_load_2d(cdst + (kBM / 2) * C::kCodePitch, &tmap_codes, st * (KSK / 8), row_b, &cfull[slot]);
+          ++issued;
           if (++slot == cst) { slot = 0; if (!lap0) ph ^= 1u; lap0 = false; }
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
     }
     if (!ok) fail(lane);
+    // After an abort the consumers stop waiting on the stages in flight: wait (bounded) until the
+    // copies of the last cst stages issued have landed, so none lands after the CTA has exited.
+    // Stage i used slot i % cst and completes phase (i / cst) of that slot's full barrier.
+    if (lane == 0 && *abort_flag)
+      for (int64_t i = issued > cst ? issued - cst : 0; i < issued; ++i)
+        mbar_wait(&cfull[i % cst], static_cast<uint32_t>((i / cst) & 1));
     __syncwarp();
   } else if (warp == 3) {
     // ---------------------------- token producer ----------------------------
@@ -337,6 +345,7 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
       int slot = 0;
       uint32_t ph = 0;
       bool lap0 = true, ok = true;
+      int64_t issued = 0;                      // token stages issued
       for (int t = blockIdx.x; t < total && ok && !*abort_flag; t += gridDim.x) {
         Tile T;
         decode_tile(A, table, offs, t, NMAX, T);
@@ -348,10 +357,14 @@ tm_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
 #pragma unroll
           for (int sub = 0; sub < C::kSubs; ++sub)
             tma_load_2d(tdst + sub * C::kTokSub, &tmap_tok, st * KSK + 64 * sub, r0, &tfull[slot]);
+          ++issued;
           if (++slot == TSTAGES) { slot = 0; if (!lap0) ph ^= 1u; lap0 = false; }
         }
       }
       if (!ok) fail(0);
+      if (*abort_flag)                         // (as for the code stages above)
+        for (int64_t i = issued > TSTAGES ? issued - TSTAGES : 0; i < issued; ++i)
+          mbar_wait(&tfull[i % TSTAGES], static_cast<uint32_t>((i / TSTAGES) & 1));
     }
     __syncwarp();
   } else if (warp == 1 || (warp >= C::kIssuerWarp0 && warp < C::kEpiWarp1)) {
