@@ -133,13 +133,14 @@ def test_golden_l1_words_through_linear(M):
 def test_workspace_cache_per_stream_and_kept_alive():
     """Scratch is shared only by calls on one stream, and an outgrown buffer stays allocated (a
     CUDA graph captured with it keeps a valid pointer)."""
-    a = api.workspace(1000, "cuda")
-    s2 = torch.cuda.Stream()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    a = api.workspace(1000, "cuda", s1)
     b = api.workspace(1000, "cuda", s2)
     assert a.data_ptr() != b.data_ptr()
+    assert api.workspace(500, "cuda", s1) is a
     ptr_a = a.data_ptr()
-    c = api.workspace(1 << 20, "cuda")          # outgrows the current stream's buffer
-    assert c.data_ptr() != ptr_a and c.numel() >= 1 << 20
-    assert api.workspace(500, "cuda") is c
-    key = (torch.device("cuda", torch.cuda.current_device()), torch.cuda.current_stream().cuda_stream)
+    c = api.workspace(a.numel() + (1 << 20), "cuda", s1)      # outgrows s1's buffer
+    assert c.data_ptr() != ptr_a and c.numel() >= a.numel() + (1 << 20)
+    assert api.workspace(500, "cuda", s1) is c
+    key = (torch.device("cuda", torch.cuda.current_device()), s1.cuda_stream)
     assert any(t.data_ptr() == ptr_a for t in api._WS[key])
