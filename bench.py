@@ -226,7 +226,7 @@ def kernel_source_hash(src="stream_gemm.cu"):
     return h.hexdigest()[:16]
 
 
-def read_profile_traffic(name, src="stream_gemm.cu"):
+def read_profile_traffic(name, src="stream_gemm.cu", key="dram_bytes_per_step"):
     """DRAM bytes of one step's grouped-GEMM launches from a committed ncu summary, if taken on
     the current kernel source (None otherwise)."""
     path = os.path.join(ROOT, "profiles", name)
@@ -240,7 +240,7 @@ def read_profile_traffic(name, src="stream_gemm.cu"):
     if vals.get("kernel_source_sha256_16") != kernel_source_hash(src):
         return None
     try:
-        return float(vals["dram_bytes_per_step"])
+        return float(vals[key])
     except (KeyError, ValueError):
         return None
 
@@ -298,7 +298,8 @@ def native_gemv(args, world, rank, local):
                    "l2": f"no flush: {nc} weight copies (264 MB) rotate"},
         "gpu_launches": 2 * calls,
         "roofline": {"bound": "hbm", "achieved": round(byts / us / 1e3, 1), "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(byts / us / 1e3 / hbm_peak, 4), "traffic": None,
+                     "frac": round(byts / us / 1e3 / hbm_peak, 4),
+                     "traffic": read_profile_traffic("stream_gemm_dense_gemv.md", key="dram_bytes_per_call"),
                      "kernel": "stream_gemm_kernel with its preparation pass", "algorithmic_bytes_per_call": byts,
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"},
     }), flush=True)
