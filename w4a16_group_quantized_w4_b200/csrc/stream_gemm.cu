@@ -121,23 +121,20 @@ static bool encode_scales_map(CUtensorMap* m, const uint16_t* scales, int64_t ro
 
 // Ring depth and offsets for one launch: each of the CTA's two pipelines gets half of the shared
 // memory left next to the unit table, with as many slots (up to kMaxStages) as fit.
-static w4::Layout make_layout(int MT, int GS, int scale_mode, int kg, int E, bool split, bool zp) {
+static w4::Layout make_layout(int MT, int GS, int scale_mode, int kg, int E, bool zp) {
   w4::Layout L{};
   L.sc_bytes = scale_mode == w4::kScaleTma ? 2 * w4::kHalf * GS * 2
              : scale_mode == w4::kScaleBlock ? 2 * w4::kHalf * kg * 2 : 0;
   L.slot_bytes = (w4::slot_sc_off(MT, GS, zp) + L.sc_bytes + 1023) & ~1023;
   const int table_bytes = (E + 1) * 12;
-  const int ep_bytes = split ? MT * w4::kEpPitch * 4 : 0;
   const int red_bytes = 2 * 4 * (MT / 8) * 2 * 32 * 16;
   const int budget = ((w4::kSmemPerCta - 1024 - table_bytes) / w4::kPipes) & ~1023;   // per pipeline
-  const int fixed = ep_bytes + red_bytes + (2 * w4::kMaxStages + 1) * 8 + 16 + 128;
+  const int fixed = red_bytes + (2 * w4::kMaxStages + 1) * 8 + 16 + 128;
   int S = (budget - fixed) / L.slot_bytes;
   if (S > w4::kMaxStages) S = w4::kMaxStages;
   L.stages = S;
   int off = S * L.slot_bytes;
-  L.ep_off = split ? off : -1;
-  off += ep_bytes;
-  L.red_off = off;                               // (16-byte aligned: slots are 1 KB, ep 16 B multiples)
+  L.red_off = off;                               // (16-byte aligned: slots are 1 KB)
   off += red_bytes;
   L.bar_off = (off + 7) & ~7;
   off = L.bar_off + (2 * S + 1) * 8;
@@ -288,7 +285,7 @@ w4_status w4_stream_setup(const uint32_t* codes, const uint16_t* scales, const i
   } else {
     scale_mode = w4::kScaleLdg;
   }
-  A.L = make_layout(p.MT, p.GS, scale_mode, A.kg, E, p.splits > 1, zp);
+  A.L = make_layout(p.MT, p.GS, scale_mode, A.kg, E, zp);
   if (A.L.stages < 2) return W4_ERR_UNSUPPORTED;
   C.A = A;
   C.p = p;

@@ -22,7 +22,6 @@ constexpr int kHalf = kBN / 2;                // rows per TMA box
 constexpr int kBoxG = 8;                      // groups per code box (128 bytes of a row)
 constexpr int kBoxBytes = kHalf * 128;        // one 64-row code box
 constexpr int kBlockMaxKg = 24;               // scale-block mode: two 64-row blocks of <= 24 groups
-constexpr int kEpPitch = kBN + 4;             // floats per token row in the epilogue buffer
 constexpr int kPB = 12;                       // preparation pass: 256-k blocks per register batch
 // dynamic shared memory of the CTA (227 KB opt-in limit per block)
 constexpr int kSmemPerCta = 232448;
@@ -55,13 +54,12 @@ __host__ __device__ constexpr int slot_desc_off(int MT, int GS, bool ZP = false)
 __host__ __device__ constexpr int slot_sc_off(int MT, int GS, bool ZP = false) { return slot_desc_off(MT, GS, ZP) + 128; }
 
 // Shared-memory layout of one launch (offsets from the 1024-byte aligned base): pipeline p's
-// ring at p * pipe_bytes, its split-K epilogue buffer, barriers and flags after the ring; then the
+// ring at p * pipe_bytes, its k-part hand-over buffer, barriers and flags after the ring; then the
 // unit table.
 struct Layout {
   int stages;
   int slot_bytes;            // one slot (multiple of 1024)
   int sc_bytes;              // scale bytes per slot
-  int ep_off;                // split-K epilogue buffer (MT x kEpPitch floats), or -1
   int red_off;               // k-part hand-over: 2 x (4 m-blocks x MT/8 x 2 tiles x 32 lanes) float4
   int bar_off;               // 2 * stages mbarriers, then the epilogue barrier
   int flag_off;              // 16 bytes
@@ -478,7 +476,6 @@ __device__ __forceinline__ void stream_gemm_body(const CUtensorMap& tmap_codes, 
 #pragma unroll
   for (int r = 0; r < 4; ++r) soff[r] = kScOff + (trow[r] >> 6) * (kHalf * GS * 2) + (trow[r] & 63) * (GS * 2);
   const uint32_t ring = smem_u32(smem);
-  float* ep = reinterpret_cast<float*>(smem + (L.ep_off >= 0 ? L.ep_off : 0));
   float4* red = reinterpret_cast<float4*>(smem + L.red_off);
   int cslot = 0;          // ring slot and mbarrier phase of the current stage
   uint32_t cphase = 0;
@@ -746,50 +743,49 @@ __device__ __forceinline__ void stream_gemm_body(const CUtensorMap& tmap_codes, 
         }
       }
     } else {
-      // split-K: float32 partials through shared memory, then the last pipeline to finish its
-      // part of the tile reduces them in split order (and applies the GELU gate)
-      if (kp == 0) {
+      // split-K: each K part writes its float32 partials straight from registers; the last
+      // pipeline to finish its part of the tile reduces them in split order (and applies the
+      // GELU gate).  One meeting puts every warp's partials before the thread that counts the
+      // arrival (its fence after the meeting covers them all), a second passes the verdict on.
+      const int ctid = warp * 32 + lane;
+      const int Nh = A.N >> 1;
+      if (kp == 0 && !flags[0]) {
+        float* pbase = A.partial + (static_cast<int64_t>(sp_last) * A.rows + r0) * A.N;
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          const int t0 = b * 8 + 2 * tq;
+        for (int i = 0; i < 2; ++i) {
+          // partial columns of this thread's rows (GELU: rows 0..63 gate j, 64..127 up j)
+          int nl, nh;
+          bool okl, okh;
+          if (gelu) {
+            const int j = nt * kHalf + 16 * mb + 8 * i + gid;
+            okl = okh = j < Nh;
+            nl = j;
+            nh = Nh + j;
+          } else {
+            nl = nt * kBN + trow[2 * i];
+            nh = nt * kBN + trow[2 * i + 1];
+            okl = nl < A.N;
+            okh = nh < A.N;
+          }
 #pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int rl = trow[2 * i], rh = trow[2 * i + 1];
-            ep[t0 * kEpPitch + rl] = acc[b][i][0];
-            ep[(t0 + 1) * kEpPitch + rl] = acc[b][i][1];
-            ep[t0 * kEpPitch + rh] = acc[b][i][2];
-            ep[(t0 + 1) * kEpPitch + rh] = acc[b][i][3];
+          for (int b = 0; b < NB; ++b) {
+            const int t0 = b * 8 + 2 * tq;
+            if (t0 < mt) {
+              if (okl) pbase[static_cast<int64_t>(t0) * A.N + nl] = acc[b][i][0];
+              if (okh) pbase[static_cast<int64_t>(t0) * A.N + nh] = acc[b][i][2];
+            }
+            if (t0 + 1 < mt) {
+              if (okl) pbase[static_cast<int64_t>(t0 + 1) * A.N + nl] = acc[b][i][1];
+              if (okh) pbase[static_cast<int64_t>(t0 + 1) * A.N + nh] = acc[b][i][3];
+            }
           }
         }
       }
       if (!epi_sync()) return;
-      const int ctid = warp * 32 + lane;
-      const int Nh = A.N >> 1;
-      // partial column of tile row c (GELU: rows 0..63 gate j, 64..127 up j of outputs j)
-      auto pcol = [&](int c, bool& ok) -> int {
-        if (gelu) {
-          const int j = nt * kHalf + (c & (kHalf - 1));
-          ok = j < Nh;
-          return c < kHalf ? j : Nh + j;
-        }
-        const int n = nt * kBN + c;
-        ok = n < A.N;
-        return n;
-      };
-      if (!flags[0]) {
-        for (int idx = ctid; idx < mt * kBN; idx += kWarps * 32) {
-          const int t = idx / kBN, c = idx % kBN;
-          bool ok;
-          const int n = pcol(c, ok);
-          if (ok)
-            A.partial[(static_cast<int64_t>(sp_last) * A.rows + r0 + t) * A.N + n] = ep[t * kEpPitch + c];
-        }
-      }
-      __threadfence();
-      if (!epi_sync()) return;
       if (ctid == 0) {
         int is_last = 0;
         if (!flags[0]) {
+          __threadfence();
           const int prev = atomicAdd(&A.counters[tile_last], 1);
           is_last = (prev == A.splits - 1);
           if (is_last) A.counters[tile_last] = 0;
@@ -828,10 +824,14 @@ __device__ __forceinline__ void stream_gemm_body(const CUtensorMap& tmap_codes, 
           }
         }
       }
-      if (!epi_sync()) return;
-      if (HO && A.tile_done && flags[1] && ctid == 0) {
-        __threadfence();
-        atomicAdd(A.tile_done + blk_last, 1);
+      // (flags[1] is next written two meetings into the next split unit, after every warp has
+      // read it here)
+      if (HO && A.tile_done) {
+        if (!epi_sync()) return;
+        if (flags[1] && ctid == 0) {
+          __threadfence();
+          atomicAdd(A.tile_done + blk_last, 1);
+        }
       }
     }
 #pragma unroll
