@@ -180,7 +180,7 @@ moe_layer_kernel(const __grid_constant__ CUtensorMap gu_tmap, const __grid_const
                                            const_cast<uint8_t*>(P.gu.xw), P.gu.n_stages, P.n_blocks, P.dev_status,
                                            h, static_cast<int64_t>(cw) * G + rb, ncw);
     };
-    stream_gemm_body<8, 16, true, SGU, false, true>(gu_tmap, gu_smap, P.gu, smem_raw, pre_gu);
+    stream_gemm_body<8, 16, true, SGU, false, 2, true>(gu_tmap, gu_smap, P.gu, smem_raw, pre_gu);
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) stream_gemm_inval(P.gu.L, smem_raw);
@@ -192,7 +192,7 @@ moe_layer_kernel(const __grid_constant__ CUtensorMap gu_tmap, const __grid_const
                                            const_cast<uint8_t*>(P.dn.xw), P.dn.n_stages, P.n_blocks, P.dev_status,
                                            h, static_cast<int64_t>(cw) * G + rb, ncw);
     };
-    stream_gemm_body<8, 16, false, SDN, false, true>(dn_tmap, dn_smap, P.dn, smem_raw, pre_dn);
+    stream_gemm_body<8, 16, false, SDN, false, 2, true>(dn_tmap, dn_smap, P.dn, smem_raw, pre_dn);
     __syncthreads();
     if (tid == 0) stream_gemm_inval(P.dn.L, smem_raw);
     __syncthreads();

@@ -49,27 +49,27 @@
 #include "stream_gemm.cuh"
 
 namespace w4 {
-template <int MT, int GS, bool GELU, int SCALE, bool ZP>
+template <int MT, int GS, bool GELU, int SCALE, bool ZP, int SPL>
 __global__ void __launch_bounds__(kThreads, 1)
 stream_gemm_kernel(const __grid_constant__ CUtensorMap tmap_codes,
                    const __grid_constant__ CUtensorMap tmap_scales, const __grid_constant__ StreamArgs A) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  stream_gemm_body<MT, GS, GELU, SCALE, ZP>(tmap_codes, tmap_scales, A, smem_raw);
+  stream_gemm_body<MT, GS, GELU, SCALE, ZP, SPL>(tmap_codes, tmap_scales, A, smem_raw);
 }
 
-template <int MT, int GS, bool ZP>
+template <int MT, int GS, bool ZP, bool CHUNK>
 __global__ void __launch_bounds__(256)
 stream_prep_kernel(const uint16_t* __restrict__ a, const int32_t* __restrict__ a_row_of_pair, int k_div,
                    int64_t a_rows, int64_t rows, int K, const int32_t* __restrict__ offsets, int E,
                    uint8_t* __restrict__ xw, int n_stages, int64_t n_blocks, int32_t* __restrict__ counters,
-                   int n_counters, int32_t* dev_status) {
+                   int n_counters, int32_t* dev_status, int bchunk) {
   extern __shared__ int prep_smem[];
   // The GEMM after this pass may launch only once the kernels before the pass have completed
   // (it reads the routing and starts its weight stream before waiting for this pass).
   pdl_wait();
   pdl_trigger();
-  stream_prep_body<MT, GS, ZP>(a, a_row_of_pair, k_div, a_rows, rows, K, offsets, E, xw, n_stages, n_blocks,
-                               counters, n_counters, dev_status, prep_smem);
+  stream_prep_body<MT, GS, ZP, false, CHUNK>(a, a_row_of_pair, k_div, a_rows, rows, K, offsets, E, xw, n_stages,
+                                             n_blocks, counters, n_counters, dev_status, prep_smem, bchunk);
 }
 
 }  // namespace w4
@@ -206,41 +206,60 @@ size_t w4_stream_workspace_bytes(int64_t rows, int N, int K, int E, int epi, boo
   return b;
 }
 
-template <int MT, int GS, bool GELU, int SCALE, bool ZP>
+template <int MT, int GS, bool GELU, int SCALE, bool ZP, int SPL>
 static w4_status launch_one(const CUtensorMap& tmap, const CUtensorMap& smap, const w4::StreamArgs& A,
                             int sm_count, cudaStream_t stream) {
   static int attr_done[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(w4::stream_gemm_kernel<MT, GS, GELU, SCALE, ZP>,
+    if (cudaFuncSetAttribute(w4::stream_gemm_kernel<MT, GS, GELU, SCALE, ZP, SPL>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, w4::kSmemPerCta) != cudaSuccess)
       return W4_ERR_CUDA;
     attr_done[dev] = 1;
   }
-  return launch_pdl(w4::stream_gemm_kernel<MT, GS, GELU, SCALE, ZP>, dim3(sm_count), dim3(w4::kThreads),
+  return launch_pdl(w4::stream_gemm_kernel<MT, GS, GELU, SCALE, ZP, SPL>, dim3(sm_count), dim3(w4::kThreads),
                     A.L.total, stream, tmap, smap, A) == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+template <int MT, int GS, bool GELU, int SCALE, bool ZP>
+static w4_status launch_split(const CUtensorMap& tmap, const CUtensorMap& smap, const w4::StreamArgs& A,
+                              int sm_count, cudaStream_t stream) {
+  return A.splits > 1 ? launch_one<MT, GS, GELU, SCALE, ZP, 1>(tmap, smap, A, sm_count, stream)
+                      : launch_one<MT, GS, GELU, SCALE, ZP, 0>(tmap, smap, A, sm_count, stream);
 }
 
 template <int MT, int GS, bool GELU>
 static w4_status launch_scale(int scale_mode, bool zp, const CUtensorMap& tmap, const CUtensorMap& smap,
                               const w4::StreamArgs& A, int sm_count, cudaStream_t stream) {
-  if (zp) return launch_one<MT, GS, GELU, w4::kScaleLdg, true>(tmap, smap, A, sm_count, stream);
-  if (scale_mode == w4::kScaleTma) return launch_one<MT, GS, GELU, w4::kScaleTma, false>(tmap, smap, A, sm_count, stream);
-  if (scale_mode == w4::kScaleBlock) return launch_one<MT, GS, GELU, w4::kScaleBlock, false>(tmap, smap, A, sm_count, stream);
-  return launch_one<MT, GS, GELU, w4::kScaleLdg, false>(tmap, smap, A, sm_count, stream);
+  if (zp) return launch_split<MT, GS, GELU, w4::kScaleLdg, true>(tmap, smap, A, sm_count, stream);
+  if (scale_mode == w4::kScaleTma) return launch_split<MT, GS, GELU, w4::kScaleTma, false>(tmap, smap, A, sm_count, stream);
+  if (scale_mode == w4::kScaleBlock) return launch_split<MT, GS, GELU, w4::kScaleBlock, false>(tmap, smap, A, sm_count, stream);
+  return launch_split<MT, GS, GELU, w4::kScaleLdg, false>(tmap, smap, A, sm_count, stream);
+}
+
+template <int MT, int GS, bool ZP>
+static cudaError_t launch_prep_z(dim3 grid, size_t smem, cudaStream_t stream, const uint16_t* a,
+                                 const int32_t* a_row_of_pair, int kd, int64_t a_rows, int64_t rows, int K,
+                                 const int32_t* offsets, int E, uint8_t* xw, int n_stages, int64_t n_blocks,
+                                 int32_t* counters, int n_counters, int32_t* dev_status, int bchunk, bool chunk) {
+  if (chunk)
+    return launch_pdl(w4::stream_prep_kernel<MT, GS, ZP, true>, grid, dim3(256), smem, stream, a, a_row_of_pair, kd,
+                      a_rows, rows, K, offsets, E, xw, n_stages, n_blocks, counters, n_counters, dev_status, bchunk);
+  return launch_pdl(w4::stream_prep_kernel<MT, GS, ZP, false>, grid, dim3(256), smem, stream, a, a_row_of_pair, kd,
+                    a_rows, rows, K, offsets, E, xw, n_stages, n_blocks, counters, n_counters, dev_status, bchunk);
 }
 
 template <int MT, int GS>
 static cudaError_t launch_prep(bool zp, dim3 grid, size_t smem, cudaStream_t stream, const uint16_t* a,
                                const int32_t* a_row_of_pair, int kd, int64_t a_rows, int64_t rows, int K,
                                const int32_t* offsets, int E, uint8_t* xw, int n_stages, int64_t n_blocks,
-                               int32_t* counters, int n_counters, int32_t* dev_status) {
+                               int32_t* counters, int n_counters, int32_t* dev_status, int bchunk, bool chunk) {
   if (zp)
-    return launch_pdl(w4::stream_prep_kernel<MT, GS, true>, grid, dim3(256), smem, stream, a, a_row_of_pair, kd,
-                      a_rows, rows, K, offsets, E, xw, n_stages, n_blocks, counters, n_counters, dev_status);
-  return launch_pdl(w4::stream_prep_kernel<MT, GS, false>, grid, dim3(256), smem, stream, a, a_row_of_pair, kd,
-                    a_rows, rows, K, offsets, E, xw, n_stages, n_blocks, counters, n_counters, dev_status);
+    return launch_prep_z<MT, GS, true>(grid, smem, stream, a, a_row_of_pair, kd, a_rows, rows, K, offsets, E, xw,
+                                       n_stages, n_blocks, counters, n_counters, dev_status, bchunk, chunk);
+  return launch_prep_z<MT, GS, false>(grid, smem, stream, a, a_row_of_pair, kd, a_rows, rows, K, offsets, E, xw,
+                                      n_stages, n_blocks, counters, n_counters, dev_status, bchunk, chunk);
 }
 
 w4_status w4_stream_setup(const uint32_t* codes, const uint16_t* scales, const int32_t* offsets, int E,
@@ -334,16 +353,23 @@ w4_status w4_launch_stream_gemm(const uint16_t* a, const int32_t* a_row_of_pair,
     // (the preparation pass clears the split-K arrival counters)
     const int kd = k_div > 0 ? k_div : 1;
     const int64_t a_rows = a_row_of_pair ? rows / kd : rows;
-    const int64_t wblocks = (rows + 7) / 8;
+    // A few rows (GEMVs, one-token decode) are cut into pieces of bchunk 256-k blocks, one warp
+    // each (every piece finds the row's exponent itself), so that about 256 warps share the
+    // conversion instead of one warp per row working through it alone.
+    const int nblk = p.n_stages * (p.GS / w4::kBoxG);
+    const int64_t want = rows >= 256 ? 1 : std::min<int64_t>(nblk, 256 / rows);
+    const int bchunk = static_cast<int>((nblk + want - 1) / want);
+    const int64_t items = rows * ((nblk + bchunk - 1) / bchunk);
+    const int64_t wblocks = (items + 7) / 8;
     const int grid = static_cast<int>(wblocks < 16LL * sm_count ? wblocks : 16LL * sm_count);
     const int n_counters = static_cast<int>(C.counters_bytes / sizeof(int32_t));
     const size_t psmem = dense ? 0 : static_cast<size_t>(E + 1) * 2 * sizeof(int);
     const int32_t* offs = dense ? nullptr : offsets;
     const cudaError_t e = p.MT == 8
         ? launch_prep<8, 16>(zp, dim3(grid), psmem, stream, a, a_row_of_pair, kd, a_rows, rows, K, offs, E, wsb,
-                             p.n_stages, C.n_blocks, C.A.counters, n_counters, dev_status)
+                             p.n_stages, C.n_blocks, C.A.counters, n_counters, dev_status, bchunk, bchunk < nblk)
         : launch_prep<16, 8>(zp, dim3(grid), psmem, stream, a, a_row_of_pair, kd, a_rows, rows, K, offs, E, wsb,
-                             p.n_stages, C.n_blocks, C.A.counters, n_counters, dev_status);
+                             p.n_stages, C.n_blocks, C.A.counters, n_counters, dev_status, bchunk, bchunk < nblk);
     if (e != cudaSuccess) return W4_ERR_CUDA;
   }
   const bool gelu = epi == W4_EPI_GELU_GATE;

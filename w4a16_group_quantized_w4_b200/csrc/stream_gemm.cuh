@@ -193,11 +193,13 @@ struct NoPreWork {
 
 // The kernel's body (stream_gemm_kernel, and two phases of the fused MoE decode kernel): smem_raw
 // is the dynamic shared memory of the CTA.  HO: the in-kernel hand-over through A.act_ready /
-// A.tile_done is compiled in.  pre(offs, blk, w, n) runs on the n = 16 compute warps (w = 0..15)
+// A.tile_done is compiled in.  SPL: the epilogue for units without a K split (0), with one (1),
+// or either, chosen by A.splits at run time (2); the stand-alone kernel is instantiated per case
+// so that each carries only the epilogue it runs.  pre(offs, blk, w, n) runs on the n = 16 compute warps (w = 0..15)
 // once the unit table is built and before they consume the first stage, while the producers
 // already stream weights: offs / blk are the table's per-expert row offsets and first token
 // blocks (shared memory).  It may use warp-level synchronisation only.
-template <int MT, int GS, bool GELU, int SCALE, bool ZP, bool HO = false, typename Pre = NoPreWork>
+template <int MT, int GS, bool GELU, int SCALE, bool ZP, int SPL = 2, bool HO = false, typename Pre = NoPreWork>
 __device__ __forceinline__ void stream_gemm_body(const CUtensorMap& tmap_codes, const CUtensorMap& tmap_scales,
                                                  const StreamArgs& A, uint8_t* smem_raw, const Pre& pre = Pre{}) {
   constexpr int kActOff = slot_act_off(GS);
@@ -652,7 +654,7 @@ __device__ __forceinline__ void stream_gemm_body(const CUtensorMap& tmap_codes, 
     const bool last = dflags & kDescLast;
     int sp_last = 0, tile_last = 0, blk_last = 0;   // the unit's K split, tile id, token block
     if (last) {
-      if (A.splits > 1 || HO) {
+      if ((SPL == 2 ? A.splits > 1 : SPL == 1) || HO) {
         const int4 d1 = *reinterpret_cast<const int4*>(sp8 + kDescOff + 16);   // before the slot is freed
         sp_last = d1.y;
         tile_last = d1.z;
@@ -701,7 +703,7 @@ __device__ __forceinline__ void stream_gemm_body(const CUtensorMap& tmap_codes, 
           acc[b][i][0] += v.x; acc[b][i][1] += v.y; acc[b][i][2] += v.z; acc[b][i][3] += v.w;
         }
     }
-    if (A.splits == 1) {
+    if (SPL == 2 ? A.splits == 1 : SPL == 0) {
       // straight from registers: the k-part 0 thread holds rows rlo / rhi of both tiles for tokens
       // 2tq, 2tq + 1 of each block
       if (kp == 0) {
@@ -871,14 +873,18 @@ struct PrepHooks {
   uint64_t wait_ns;
 };
 
-// The rows [wfirst, rows) in steps of wstride, one warp each: offs / blk are the per-expert row
-// offsets and first token blocks (grouped), held in shared memory.
-template <int MT, int GS, bool ZP, bool INK>
+// Work items [wfirst, rows * nchunk) in steps of wstride, one warp each: item w is row
+// w / nchunk, 256-k blocks [c * bchunk, (c + 1) * bchunk) with c = w % nchunk (every item finds
+// the row's exponent over the whole row; CHUNK = false compiles whole rows only, which the
+// hand-over hooks require).  offs / blk are the per-expert row offsets and first token blocks
+// (grouped), held in shared memory.
+template <int MT, int GS, bool ZP, bool INK, bool CHUNK = false>
 __device__ __forceinline__ void stream_prep_rows(const uint16_t* __restrict__ a, const int32_t* __restrict__ a_row_of_pair,
                                                  int k_div, int64_t a_rows, int64_t rows, int K, bool grouped,
                                                  const int* offs, const int* blk, int E, uint8_t* __restrict__ xw,
                                                  int n_stages, int64_t n_blocks, int32_t* dev_status,
-                                                 const PrepHooks& hk, int64_t wfirst, int64_t wstride) {
+                                                 const PrepHooks& hk, int64_t wfirst, int64_t wstride,
+                                                 int bchunk = 1 << 20) {
   constexpr int kRec = rec_bytes(MT, GS, ZP);
   constexpr int kXP = rec_xp(GS);
   constexpr int kQOff = rec_qoff(MT, GS);
@@ -888,7 +894,12 @@ __device__ __forceinline__ void stream_prep_rows(const uint16_t* __restrict__ a,
   const int lane = threadIdx.x & 31;
   const int nv = K >> 3;                          // 8-element chunks in the row
   const int nblk = n_stages * kBPS;               // 256-k blocks written (zeros past K)
-  for (int64_t r = wfirst; r < rows; r += wstride) {
+  if (bchunk > nblk) bchunk = nblk;
+  const int nchunk = CHUNK ? (nblk + bchunk - 1) / bchunk : 1;
+  for (int64_t w = wfirst; w < rows * nchunk; w += wstride) {
+    const int64_t r = CHUNK ? w / nchunk : w;
+    const int jb0 = CHUNK ? static_cast<int>(w - r * nchunk) * bchunk : 0;   // this item's blocks
+    const int jb1 = !CHUNK ? nblk : (jb0 + bchunk < nblk ? jb0 + bchunk : nblk);
     int64_t src = r;
     if (a_row_of_pair) {
       src = (INK ? __ldcg(a_row_of_pair + r) : __ldg(a_row_of_pair + r)) / k_div;
@@ -948,18 +959,18 @@ __device__ __forceinline__ void stream_prep_rows(const uint16_t* __restrict__ a,
     const int f = shift_for(m, 14);
     const float m1 = pow2f(f), m16 = pow2f(f - 4);
     uint8_t* rec0 = xw + b * n_stages * kRec;
-    for (int j0 = 0; j0 < nblk; j0 += kPB) {
-      if (nblk > kPB) {                          // long rows: the batch again (from L1 / L2)
+    for (int j0 = jb0; j0 < jb1; j0 += kPB) {
+      if (nblk > kPB || (CHUNK && jb0 > 0)) {    // the batch again (from L1 / L2)
 #pragma unroll
         for (int t = 0; t < kPB; ++t) {
           const int i = (j0 + t) * 32 + lane;
-          v[t] = i < nv ? ld_row(i) : make_uint4(0, 0, 0, 0);
+          v[t] = i < nv && j0 + t < jb1 ? ld_row(i) : make_uint4(0, 0, 0, 0);
         }
       }
 #pragma unroll
       for (int t = 0; t < kPB; ++t) {
         const int j = j0 + t;
-        if (j >= nblk) break;
+        if (j >= jb1) break;
         const uint32_t w[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
         uint32_t h[4];
         f16_pairs_l1(w, m1, m16, h);             // (x0, x4), (x1, x5)/16, (x2, x6), (x3, x7)/16
@@ -988,8 +999,10 @@ __device__ __forceinline__ void stream_prep_rows(const uint16_t* __restrict__ a,
         }
       }
     }
+    // the row's multiplier in every stage whose first block is this item's
     for (int j = lane; j < n_stages; j += 32)
-      *reinterpret_cast<float*>(rec0 + static_cast<int64_t>(j) * kRec + kMOff + slot * 4) = pow2f(-f);
+      if (!CHUNK || (j * kBPS >= jb0 && j * kBPS < jb1))
+        *reinterpret_cast<float*>(rec0 + static_cast<int64_t>(j) * kRec + kMOff + slot * 4) = pow2f(-f);
     if (hk.ready) {
       // the records are read by bulk copies (the async proxy) of other CTAs; the release is made
       // once for the warp's writes, after the warp has met
@@ -1003,13 +1016,13 @@ __device__ __forceinline__ void stream_prep_rows(const uint16_t* __restrict__ a,
   }
 }
 
-template <int MT, int GS, bool ZP, bool INK = false>
+template <int MT, int GS, bool ZP, bool INK = false, bool CHUNK = false>
 __device__ __forceinline__ void stream_prep_body(const uint16_t* __restrict__ a, const int32_t* __restrict__ a_row_of_pair,
                                                  int k_div, int64_t a_rows, int64_t rows, int K,
                                                  const int32_t* __restrict__ offsets, int E, uint8_t* __restrict__ xw,
                                                  int n_stages, int64_t n_blocks, int32_t* __restrict__ counters,
                                                  int n_counters, int32_t* dev_status, int* prep_smem,
-                                                 const PrepHooks& hk = PrepHooks{}) {
+                                                 int bchunk = 1 << 20, const PrepHooks& hk = PrepHooks{}) {
   int* offs = prep_smem;                          // [E + 1]
   int* blk = prep_smem + (E + 1);                 // [E + 1]
   const int lane = threadIdx.x & 31;
@@ -1043,9 +1056,9 @@ __device__ __forceinline__ void stream_prep_body(const uint16_t* __restrict__ a,
     }
     __syncthreads();
   }
-  stream_prep_rows<MT, GS, ZP, INK>(a, a_row_of_pair, k_div, a_rows, rows, K, offsets != nullptr, offs, blk, E, xw,
+  stream_prep_rows<MT, GS, ZP, INK, CHUNK>(a, a_row_of_pair, k_div, a_rows, rows, K, offsets != nullptr, offs, blk, E, xw,
                                     n_stages, n_blocks, dev_status, hk, blockIdx.x * wpb + (threadIdx.x >> 5),
-                                    gridDim.x * wpb);
+                                    gridDim.x * wpb, bchunk);
 }
 
 }  // namespace w4
