@@ -524,8 +524,14 @@ def native(args, world, rank, local):
         secondary = run_secondary(args, device, stream)
 
     cpu_base = None
+    parity = None
     if rank == 0 and world == 1:
-        cpu_base = cpu_baseline(case)
+        with torch.cuda.stream(stream):
+            y_dev = layers[0](x, logits).float().cpu().numpy()
+        stream.synchronize()
+        ref = {}
+        cpu_base = cpu_baseline(case, ref)
+        parity = parity_stats(y_dev, ref, rt)
 
     del graph                    # (holds no collective) released before the group goes
     ranks_finish(world)
@@ -557,6 +563,7 @@ def native(args, world, rank, local):
         "step_time_distribution": step_dist,
         "roofline": roofline,
         "cpu_baseline": cpu_base,
+        "parity": parity,
         "secondary": secondary,
     }
     print(json.dumps(line), flush=True)
@@ -571,8 +578,9 @@ def _physical_gpu_index(local):
     return local
 
 
-def cpu_baseline(case):
-    """The oracle as it stands on a bounded sample of the same workload (host cores)."""
+def cpu_baseline(case, outputs=None):
+    """The oracle as it stands on a bounded sample of the same workload (host cores).  When
+    `outputs` is a dict, it receives the sampled tokens, their oracle outputs and the routing."""
     import numpy as np
 
     from oracle import moe
@@ -584,12 +592,19 @@ def cpu_baseline(case):
     # chunks of 8 tokens until about 10 s of host work (at most every token of the layer)
     done, chunk, budget_s = 0, 8, 10.0
     t0 = time.perf_counter()
+    ys = []
     while done < case.T and time.perf_counter() - t0 < budget_s:
         tokens = np.arange(done, min(done + chunk, case.T))
-        moe.moe_layer(case.x, case.logits, case.gu_codes, case.gu_scales, case.dn_codes, case.dn_scales,
-                      case.k, tokens=tokens)
+        res = moe.moe_layer(case.x, case.logits, case.gu_codes, case.gu_scales, case.dn_codes, case.dn_scales,
+                            case.k, tokens=tokens)
+        if outputs is not None:
+            ys.append(res.y[tokens])
+            outputs["routing"] = res.routing
         done += len(tokens)
     dt = time.perf_counter() - t0
+    if outputs is not None:
+        outputs["tokens"] = np.arange(done)
+        outputs["y"] = np.concatenate(ys) if ys else np.zeros((0, case.H))
     # the same oracle on one host thread, on the first chunk only
     one = None
     try:
@@ -606,6 +621,35 @@ def cpu_baseline(case):
             "sample": f"{done} of {case.T} tokens of the same layer in chunks of {chunk} (routing of "
                       f"all {case.T} each chunk); {dt:.1f} s of float64 numpy on the host; "
                       f"value_1_thread: the first chunk with the BLAS pool limited to one thread"}
+
+
+def parity_stats(y_dev, ref, rt_dev=None):
+    """Parity of the device's layer output with the oracle's on the cpu_baseline sample: per token
+    row rel-L2 and max-abs error (as a fraction of the row's max |ref|) against the tolerance, and
+    the routing compared bit for bit over every token."""
+    import numpy as np
+    tok = ref["tokens"]
+    if tok.size == 0:
+        return None
+    y = np.asarray(y_dev, dtype=np.float64)[tok]
+    r = np.asarray(ref["y"], dtype=np.float64)
+    nref = np.linalg.norm(r, axis=1)
+    rel = np.linalg.norm(y - r, axis=1) / np.where(nref > 0, nref, 1.0)
+    mref = np.abs(r).max(axis=1)
+    mabs = np.abs(y - r).max(axis=1) / np.where(mref > 0, mref, 1.0)
+    ok = (rel <= 5e-3) & (mabs <= 2e-2)
+    out = {"tokens_checked": int(tok.size), "max_rel_l2": float(f"{rel.max():.3e}"),
+           "median_rel_l2": float(f"{np.median(rel):.3e}"), "max_abs_frac": float(f"{mabs.max():.3e}"),
+           "rows_within_tolerance": int(ok.sum()), "tolerance": {"rel_l2": 5e-3, "max_abs_frac": 2e-2},
+           "reference": "the CPU oracle (float64) on the cpu_baseline sample"}
+    if rt_dev is not None and "routing" in ref:
+        ro = ref["routing"]
+        out["routing_bit_exact"] = {
+            "topk_ids": bool(np.array_equal(rt_dev.topk_ids.cpu().numpy(), ro.topk_ids)),
+            "expert_offsets": bool(np.array_equal(rt_dev.expert_offsets.cpu().numpy(), ro.expert_offsets)),
+            "sorted_pair": bool(np.array_equal(rt_dev.sorted_pair.cpu().numpy(), ro.sorted_pair)),
+            "pair_pos": bool(np.array_equal(rt_dev.pair_pos.cpu().numpy(), ro.pair_pos))}
+    return out
 
 
 def run_secondary(args, device, stream):
