@@ -4,7 +4,20 @@
 #include <cstdint>
 #include <cstring>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/w4a16.h"
+
+// A named profiler range around each entry point, so that a timeline (nsys, ncu's NVTX filters)
+// shows the library's calls by name; without a profiler attached the calls do nothing.
+namespace {
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+  Range(const Range&) = delete;
+  Range& operator=(const Range&) = delete;
+};
+}  // namespace
 
 // kernel launchers (repack.cu, route.cu, stream_gemm.cu)
 w4_status w4_launch_repack(const uint16_t* w, int64_t groups, uint32_t* codes, uint16_t* scales,
@@ -153,6 +166,7 @@ size_t w4_workspace_bytes(int32_t op, int64_t M_or_T, int64_t N, int64_t K, int3
 
 w4_status w4_repack(const uint16_t* w, int64_t rows, int64_t K, uint32_t* codes, uint16_t* scales,
                     uint8_t* group_m, unsigned long long* off_grid_count, void* stream) {
+  const Range range("w4_repack");
   if (rows < 0 || K < 32 || K % 32) return W4_ERR_INVALID_ARG;
   if (rows > 0 && (!w || !codes || !scales)) return W4_ERR_INVALID_ARG;
   if ((w && !aligned(w, 16)) || (codes && !aligned(codes, 16)) || (scales && !aligned(scales, 2)))
@@ -166,6 +180,7 @@ w4_status w4_repack(const uint16_t* w, int64_t rows, int64_t K, uint32_t* codes,
 w4_status w4a16_linear(const uint16_t* x, const uint32_t* codes, const uint16_t* scales,
                        uint16_t* y, int64_t M, int64_t N, int64_t K, void* workspace,
                        size_t workspace_bytes, void* stream) {
+  const Range range("w4a16_linear");
   if (M < 0 || N < 1 || K < 32 || K % 32 || N > (1LL << 30) || K > (1LL << 30)) return W4_ERR_INVALID_ARG;
   if (M > 0 && (!x || !y)) return W4_ERR_INVALID_ARG;
   if (!codes || !scales) return W4_ERR_INVALID_ARG;
@@ -187,6 +202,7 @@ w4_status moe_route_permute(const float* logits, int32_t T, int32_t E, int32_t k
                             float* topk_w, int32_t* expert_offsets, int32_t* sorted_pair,
                             int32_t* pair_pos, void* workspace, size_t workspace_bytes,
                             void* stream) {
+  const Range range("moe_route_permute");
   if (T < 0 || E < 1 || E > 1024 || k < 1 || k > 32 || k > E) return W4_ERR_INVALID_ARG;
   if (static_cast<int64_t>(T) * k > (1LL << 30)) return W4_ERR_UNSUPPORTED;
   if (!expert_offsets) return W4_ERR_INVALID_ARG;
@@ -201,6 +217,7 @@ w4_status moe_w4a16_gmm(const uint16_t* a, const int32_t* a_row_of_pair, int32_t
                         int32_t E, int64_t rows, int32_t N, int32_t K, int32_t epilogue,
                         uint16_t* out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
                         void* stream) {
+  const Range range("moe_w4a16_gmm");
   if (E < 1 || E > 1024 || rows < 0 || N < 1 || K < 32 || K % 32) return W4_ERR_INVALID_ARG;
   if (epilogue != W4_EPI_NONE && epilogue != W4_EPI_GELU_GATE) return W4_ERR_INVALID_ARG;
   if (epilogue == W4_EPI_GELU_GATE && (N % 2)) return W4_ERR_INVALID_ARG;
@@ -229,6 +246,7 @@ w4_status w4_testing_stream_gmm_stall(const uint16_t* a, const int32_t* a_row_of
                                       int32_t K, int32_t epilogue, uint16_t* out, void* workspace,
                                       size_t workspace_bytes, int32_t* dev_status, void* stream,
                                       uint64_t wait_ns, int32_t stall_after) {
+  const Range range("w4_testing_stream_gmm_stall");
   if (E < 1 || E > 1024 || rows < 0 || N < 1 || K < 32 || K % 32 || !codes || !scales || !expert_offsets)
     return W4_ERR_INVALID_ARG;
   if (epilogue != W4_EPI_NONE && epilogue != W4_EPI_GELU_GATE) return W4_ERR_INVALID_ARG;
@@ -250,6 +268,7 @@ static bool group_ok(int64_t group, int64_t K) {
 w4_status w4a16_linear_g(const uint16_t* x, const uint32_t* codes, const uint16_t* scales,
                          const uint8_t* zeros, int32_t group, uint16_t* y, int64_t M, int64_t N, int64_t K,
                          void* workspace, size_t workspace_bytes, void* stream) {
+  const Range range("w4a16_linear_g");
   if (M < 0 || N < 1 || K < 32 || K % 32 || N > (1LL << 30) || K > (1LL << 30)) return W4_ERR_INVALID_ARG;
   if (!group_ok(group, K)) return W4_ERR_INVALID_ARG;
   if (M > 0 && (!x || !y)) return W4_ERR_INVALID_ARG;
@@ -269,6 +288,7 @@ w4_status moe_w4a16_gmm_g(const uint16_t* a, const int32_t* a_row_of_pair, int32
                           int32_t group, const int32_t* expert_offsets, int32_t E, int64_t rows,
                           int32_t N, int32_t K, int32_t epilogue, uint16_t* out, void* workspace,
                           size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  const Range range("moe_w4a16_gmm_g");
   if (E < 1 || E > 1024 || rows < 0 || N < 1 || K < 32 || K % 32) return W4_ERR_INVALID_ARG;
   if (!group_ok(group, K)) return W4_ERR_INVALID_ARG;
   if (epilogue != W4_EPI_NONE && epilogue != W4_EPI_GELU_GATE) return W4_ERR_INVALID_ARG;
@@ -289,6 +309,7 @@ w4_status moe_w4a16_layer(const uint16_t* x, const float* logits, int32_t T, int
                           const uint32_t* gu_codes, const uint16_t* gu_scales, const uint32_t* dn_codes,
                           const uint16_t* dn_scales, int32_t H, int32_t I, uint16_t* y, void* workspace,
                           size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  const Range range("moe_w4a16_layer");
   const w4_status chk = w4_layer_check(T, E, k, H, I);
   if (chk != W4_OK) return chk;
   if (T == 0) return W4_OK;
@@ -303,6 +324,7 @@ w4_status moe_w4a16_layer(const uint16_t* x, const float* logits, int32_t T, int
 
 w4_status moe_combine(const uint16_t* o, const float* topk_w, const int32_t* pair_pos, int32_t T,
                       int32_t k, int32_t H, uint16_t* y, void* stream) {
+  const Range range("moe_combine");
   if (T < 0 || k < 1 || H < 8 || H % 8) return W4_ERR_INVALID_ARG;
   if (T > 0 && (!o || !topk_w || !pair_pos || !y)) return W4_ERR_INVALID_ARG;
   if ((o && !aligned(o, 16)) || (y && !aligned(y, 16))) return W4_ERR_INVALID_ARG;
@@ -311,6 +333,7 @@ w4_status moe_combine(const uint16_t* o, const float* topk_w, const int32_t* pai
 
 w4_status moe_rms_chain(const uint16_t* y, int64_t T, int32_t H, float eps, uint16_t* x_next,
                         void* stream) {
+  const Range range("moe_rms_chain");
   if (T < 0 || H < 8 || H % 8 || !(eps >= 0.f) || eps > 1e30f) return W4_ERR_INVALID_ARG;
   if (T > 0 && (!y || !x_next)) return W4_ERR_INVALID_ARG;
   if ((y && !aligned(y, 16)) || (x_next && !aligned(x_next, 16))) return W4_ERR_INVALID_ARG;

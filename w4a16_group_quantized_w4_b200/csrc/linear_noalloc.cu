@@ -13,6 +13,7 @@
 // array's name is only a host-side stand-in for it); the first call on a device does that set-up,
 // so make the first call before any stream capture.  All calls share the array: two calls that
 // overlap on the GPU race on it and must be ordered by the caller (one stream, or events).
+#include <nvtx3/nvToolsExt.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -68,6 +69,8 @@ extern "C" {
 
 w4_status w4a16_linear_noalloc(const uint16_t* x, const uint32_t* codes, const uint16_t* scales,
                                uint16_t* y, int64_t M, int64_t N, int64_t K, void* stream) {
+  nvtxRangePushA("w4a16_linear_noalloc");
+  struct Pop { ~Pop() { nvtxRangePop(); } } pop;
   if (M < 0 || N < 1 || K < 32 || K % 32 || N > (1LL << 30) || K > (1LL << 30)) return W4_ERR_INVALID_ARG;
   if (M > 0 && (!x || !y)) return W4_ERR_INVALID_ARG;
   if (!codes || !scales) return W4_ERR_INVALID_ARG;
