@@ -81,3 +81,22 @@ def test_fused_layer_sizes_and_range():
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError):
         _lib.load(str(tmp_path / "nope.so"))
+
+
+def test_binding_signatures_match_the_header():
+    """The ctypes argument lists in _lib.SIGNATURES have the arity and the integer widths of the
+    declarations in include/w4a16.h (a drifted binding would pass arguments in the wrong slots)."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    decls = dict(re.findall(r"\b([A-Za-z_][A-Za-z0-9_]*)\s*\(([^;{}]*?)\)\s*;", text, flags=re.S))
+    width = {"int32_t": C.c_int32, "int64_t": C.c_int64, "size_t": C.c_size_t, "float": C.c_float}
+    for name, (_, args) in _lib.SIGNATURES.items():
+        assert name in decls, name
+        params = [p.strip() for p in decls[name].replace("\n", " ").split(",") if p.strip() and p.strip() != "void"]
+        assert len(params) == len(args), (name, len(params), len(args))
+        for p, a in zip(params, args):
+            if "*" in p:
+                assert a is C.c_void_p, (name, p)
+                continue
+            base = p.replace("const", "").split()[0]
+            if base in width:
+                assert a is width[base], (name, p, a)
